@@ -1,0 +1,150 @@
+"""ctypes binding over libfattn.so -- argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels.  There is no
+fallback: if the library is missing or cannot be loaded, every call raises.
+The names mirror the C ABI in include/fattn.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfattn.so")
+
+FATTN_OK = 0
+FATTN_ERR_INVALID_ARG = 1
+FATTN_ERR_UNSUPPORTED = 2
+FATTN_ERR_ALIGNMENT = 3
+FATTN_ERR_CUDA = 4
+FATTN_ERR_DEVICE_TIMEOUT = 5
+
+# Every symbol include/fattn.h declares (checked by the CPU test suite).
+EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_status_string",
+            "fattn_last_cuda_error", "fattn_device_status", "fattn_version")
+
+_lib = None
+
+
+class FattnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {status_string(status)} (status {status})"
+        if status == FATTN_ERR_CUDA:
+            msg += f": {last_cuda_error()}"
+        super().__init__(msg)
+
+
+def load():
+    """Open libfattn.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_attention_108_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fattn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    L.fattn_fwd.restype = i
+    L.fattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+    L.fattn_bwd.restype = i
+    L.fattn_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fattn_bwd_workspace_size.restype = sz
+    L.fattn_status_string.argtypes = [i]
+    L.fattn_status_string.restype = ctypes.c_char_p
+    L.fattn_last_cuda_error.argtypes = []
+    L.fattn_last_cuda_error.restype = ctypes.c_char_p
+    L.fattn_device_status.argtypes = [i]
+    L.fattn_device_status.restype = i
+    L.fattn_version.argtypes = []
+    L.fattn_version.restype = i
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().fattn_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> str:
+    return load().fattn_last_cuda_error().decode()
+
+
+def device_status(clear: bool = False) -> int:
+    return int(load().fattn_device_status(1 if clear else 0))
+
+
+def workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load().fattn_bwd_workspace_size(B, H, N, d))
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _shape4(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v); bf16 [B,H,N,d] in, bf16 O and fp32 LSE [B,H,N] out."""
+    B, H, N, d = _shape4(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    _check(out, "out")
+    _check(lse, "lse", torch.float32)
+    rc = load().fattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                          B, H, N, d, 1 if causal else 0, float(scale), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_fwd")
+    return out, lse
+
+
+def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
+        dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of L = sum(dO * O) for the forward that produced (o, lse)."""
+    B, H, N, d = _shape4(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    rc = load().fattn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          B, H, N, d, 1 if causal else 0, float(scale),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_bwd")
+    return dq, dk, dv

@@ -1,0 +1,257 @@
+// fattn.cu -- C ABI of libfattn (declared in include/fattn.h): argument
+// validation, TMA tensor-map encoding and kernel launches.  Everything the
+// operation computes runs in the kernels of fwd_kernel.cuh / bwd_kernels.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "fattn.h"
+
+#include "bwd_kernels.cuh"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+thread_local std::string t_last_cuda_error;
+
+int cuda_fail(cudaError_t e, const char* what) {
+  char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", what, cudaGetErrorString(e));
+  t_last_cuda_error = buf;
+  return FATTN_ERR_CUDA;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D view [rows, cols] of a row-major bf16 or fp32 tensor, box [box_rows, box_cols],
+// 128-byte swizzle when the box row is 128 bytes wide.
+int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
+             uint64_t cols, uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    t_last_cuda_error = "cuTensorMapEncodeTiled entry point not available";
+    return FATTN_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[96];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    t_last_cuda_error = buf;
+    return FATTN_ERR_CUDA;
+  }
+  return FATTN_OK;
+}
+
+int make_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int d) {
+  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, (uint64_t)d, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return FATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return FATTN_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * H * N;
+  if (rows >= (1ll << 31)) return FATTN_ERR_UNSUPPORTED;
+  if ((long long)H * B > 0x7fffffffll || N / 128 > 65535) return FATTN_ERR_UNSUPPORTED;
+  return FATTN_OK;
+}
+
+template <class K>
+int set_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return FATTN_OK;
+}
+
+template <int D, bool CAUSAL>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+               const fattn::FwdArgs& a, int BH, cudaStream_t st) {
+  auto kern = fattn::fattn_fwd_kernel<D, CAUSAL>;
+  constexpr int smem = fattn::FwdCfg<D>::SMEM;
+  if (int rc = set_smem(kern, smem)) return rc;
+  dim3 grid((unsigned)BH, (unsigned)a.num_q_tiles);
+  kern<<<grid, 256, smem, st>>>(mq, mk, mv, mo, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_fwd_kernel launch");
+  return FATTN_OK;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int D, bool CAUSAL>
+int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                const fattn::BwdArgs& a, int BH, cudaStream_t st) {
+  auto kern = fattn::fattn_bwd_dkdv_kernel<D, CAUSAL>;
+  constexpr int smem = fattn::BwdCfg<D>::SMEM;
+  if (int rc = set_smem(kern, smem)) return rc;
+  dim3 grid((unsigned)BH, (unsigned)a.num_tiles);
+  kern<<<grid, 256, smem, st>>>(mq, mk, mv, mdo, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dkdv_kernel launch");
+  return FATTN_OK;
+}
+
+template <int D>
+int launch_bwd_d(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int causal, float scale, void* workspace,
+                 cudaStream_t st) {
+  const long long rows = (long long)B * H * N;
+  char* ws = static_cast<char*>(workspace);
+  float* dvec = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
+  float* dq_acc = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+
+  {
+    constexpr int rpb = 256 / (D / 8);
+    const long long blocks = (rows + rpb - 1) / rpb;
+    fattn::fattn_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dq_acc,
+        rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_pre_kernel launch");
+  }
+  CUtensorMap mq, mk, mv, mdo;
+  if (int rc = make_bf16_tile_map(&mq, q, rows, D)) return rc;
+  if (int rc = make_bf16_tile_map(&mk, k, rows, D)) return rc;
+  if (int rc = make_bf16_tile_map(&mv, v, rows, D)) return rc;
+  if (int rc = make_bf16_tile_map(&mdo, dout, rows, D)) return rc;
+  fattn::BwdArgs a;
+  a.lse2 = lse2;
+  a.dvec = dvec;
+  a.dq_acc = dq_acc;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.N = N;
+  a.num_tiles = N / 128;
+  a.scale = scale;
+  a.scale_log2 = scale * kLog2e;
+  const int BH = B * H;
+  int rc = causal ? launch_dkdv<D, true>(mq, mk, mv, mdo, a, BH, st) : launch_dkdv<D, false>(mq, mk, mv, mdo, a, BH, st);
+  if (rc) return rc;
+  {
+    const long long n8 = rows * D / 8;
+    long long blocks = (n8 + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    fattn::fattn_bwd_dq_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), scale,
+                                                                     n8);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dq_kernel launch");
+  }
+  return FATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fattn_version(void) { return 0x000100; }
+
+const char* fattn_status_string(int status) {
+  switch (status) {
+    case FATTN_OK: return "ok";
+    case FATTN_ERR_INVALID_ARG: return "invalid argument";
+    case FATTN_ERR_UNSUPPORTED: return "unsupported shape (need d in {64,128}, N % 128 == 0)";
+    case FATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case FATTN_ERR_CUDA: return "CUDA error (see fattn_last_cuda_error)";
+    case FATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";
+    default: return "unknown status";
+  }
+}
+
+const char* fattn_last_cuda_error(void) { return t_last_cuda_error.c_str(); }
+
+int fattn_device_status(int clear) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, fattn::g_fattn_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  if (clear) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(fattn::g_fattn_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+  }
+  return v == 0 ? FATTN_OK : FATTN_ERR_DEVICE_TIMEOUT;
+}
+
+int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+              int causal, float scale, fattn_stream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FATTN_ERR_ALIGNMENT;
+
+  const uint64_t rows = (uint64_t)B * H * N;
+  CUtensorMap mq, mk, mv, mo;
+  if (int rc = make_bf16_tile_map(&mq, q, rows, d)) return rc;
+  if (int rc = make_bf16_tile_map(&mk, k, rows, d)) return rc;
+  if (int rc = make_bf16_tile_map(&mv, v, rows, d)) return rc;
+  if (int rc = make_bf16_tile_map(&mo, o, rows, d)) return rc;
+
+  fattn::FwdArgs a;
+  a.lse = lse;
+  a.N = N;
+  a.num_q_tiles = N / 128;
+  a.scale_log2 = scale * kLog2e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, mo, a, BH, st)
+                             : launch_fwd<64, false>(mq, mk, mv, mo, a, BH, st);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, mo, a, BH, st)
+                : launch_fwd<128, false>(mq, mk, mv, mo, a, BH, st);
+}
+
+size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d) != FATTN_OK) return 0;
+  const size_t rows = (size_t)B * H * N;
+  return 2 * align256(rows * sizeof(float)) + align256(rows * (size_t)d * sizeof(float));
+}
+
+int fattn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+              void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
+              size_t workspace_bytes, fattn_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_shape(B, H, N, d)) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return FATTN_ERR_ALIGNMENT;
+  if (workspace_bytes < fattn_bwd_workspace_size(B, H, N, d)) return FATTN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return launch_bwd_d<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, workspace, st);
+  return launch_bwd_d<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, workspace, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+/*
+ * fattn.h -- C ABI of libfattn, a B200 (sm_100a) fused exact-attention library.
+ *
+ * Operation (forward).  For every batch b and head h, with Q, K, V each N x d
+ * ("Q, K, V are all N x d", page 3, section 3 "从CUDA原理理解注意力机制的计算瓶颈"):
+ *
+ *     s_ij  = scale * <q_i, k_j>                  (scaled QK^T, page 2 "传统注意力为何容易受 IO 限制")
+ *     s_ij  = -inf  where causal and j > i         (the mask of the same op chain; causal reading)
+ *     P     = row softmax(s)                       (exact, page 2 "二、在线 Softmax 保持精确结果")
+ *     O     = P V
+ *     LSE_i = ln sum_j exp(s_ij)                   (the softmax statistic kept for the backward,
+ *                                                   page 2 "三、融合算子减少中间张量落盘")
+ *
+ * computed as one fused, tiled kernel that never writes S or P to memory:
+ * Q/K/V tiles stream through shared memory (page 1 "三、矩阵分块", page 2 "一、用分块计算提高
+ * 片上数据复用"), the row max and row sum are kept online and earlier partial
+ * outputs are rescaled when the max grows (page 3 "4.2 在线softmax技巧").
+ *
+ * Operation (backward).  Given dO = dL/dO, recompute S and P tile by tile from
+ * Q, K and LSE (page 2 "四、反向传播选择重计算而非全量保存") and return
+ *     dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D),  D_i = sum_c dO_ic O_ic,
+ *     dQ = scale * dS K,  dK = scale * dS^T Q.
+ *
+ * Tensor layout.  q, k, v, o, dout, dq, dk, dv are bfloat16, contiguous
+ * [B, H, N, d] (d innermost, row stride d elements).  lse is float32 [B, H, N].
+ * All pointers are DEVICE pointers on the current CUDA device and must be
+ * 16-byte aligned.  Outputs must not alias inputs.
+ *
+ * Supported shapes: B, H, N >= 1; N % 128 == 0; d in {64, 128};
+ * B * H * N < 2^31.  scale must be finite (any sign).
+ *
+ * Ownership and asynchrony.  The caller allocates and owns every buffer,
+ * including the backward workspace.  The library allocates no device memory
+ * and keeps no per-call state.  Every call only enqueues work on `stream` and
+ * returns; results are valid once the stream has been synchronised.  Inputs
+ * must stay alive until then.
+ *
+ * Errors.  Arguments are validated before anything is enqueued; an invalid
+ * call returns a non-zero status and has no side effects.  A failed launch
+ * returns FATTN_ERR_CUDA.  The library never synchronises the device and never
+ * traps.  Kernels bound every wait on an on-chip barrier; a wait that runs out
+ * (a library bug, never expected) records FATTN_ERR_DEVICE_TIMEOUT in a
+ * per-device status word that fattn_device_status() reads.
+ */
+#ifndef FATTN_H_
+#define FATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fattn_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  FATTN_OK = 0,
+  FATTN_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, non-finite scale, too small workspace */
+  FATTN_ERR_UNSUPPORTED = 2,    /* d not in {64,128}, N % 128 != 0, size overflow */
+  FATTN_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
+  FATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed; see fattn_last_cuda_error() */
+  FATTN_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out */
+} fattn_status;
+
+/*
+ * Forward.  Writes o [B,H,N,d] (bf16) and lse [B,H,N] (fp32, natural log of
+ * the row sum of exp of the scaled, masked scores).
+ *   q, k, v : inputs, read only.
+ *   causal  : 0 = no mask, 1 = query i attends keys 0..i.
+ *   scale   : multiplies QK^T (usually 1/sqrt(d)).
+ */
+int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+              int B, int H, int N, int d, int causal, float scale,
+              fattn_stream_t stream);
+
+/*
+ * Bytes of device workspace fattn_bwd needs for this shape (0 for an invalid
+ * shape).  Layout inside (each part 256-byte aligned): D [B,H,N] fp32,
+ * LSE*log2(e) [B,H,N] fp32, fp32 dQ accumulator [B,H,N,d].
+ */
+size_t fattn_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward.  Inputs q, k, v, o (the forward output), dout (dL/dO) and lse (the
+ * forward statistic) are read only.  Writes dq, dk, dv (bf16, [B,H,N,d]).
+ * workspace: device memory of at least fattn_bwd_workspace_size() bytes,
+ * 256-byte aligned, owned by the caller; its contents on entry do not matter.
+ * Deterministic up to the order of fp32 additions into the dQ accumulator.
+ */
+int fattn_bwd(const void* q, const void* k, const void* v, const void* o,
+              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+              int B, int H, int N, int d, int causal, float scale,
+              void* workspace, size_t workspace_bytes, fattn_stream_t stream);
+
+/* Static, human-readable text for a status code. */
+const char* fattn_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* fattn_last_cuda_error(void);
+
+/*
+ * Reads (synchronously) the current device's kernel status word: FATTN_OK, or
+ * FATTN_ERR_DEVICE_TIMEOUT if some kernel's bounded wait ran out since the last
+ * clear.  clear != 0 resets the word.  Returns FATTN_ERR_CUDA if the read fails.
+ */
+int fattn_device_status(int clear);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int fattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FATTN_H_ */

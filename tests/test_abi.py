@@ -1,0 +1,103 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every symbol the
+header declares, and rejects bad arguments before enqueuing anything (these
+calls return from validation, so no GPU is touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_108_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fattn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fattn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.LIB_PATH):
+        from exact_attention_108_b200 import build
+        build.build()
+    return binding.load()
+
+
+def test_header_declares_the_expected_entry_points():
+    assert set(_declared_functions()) == set(binding.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert binding.status_string(s)
+    assert binding.status_string(0) == "ok"
+    assert lib.fattn_version() == 0x000100
+
+
+P = 1 << 20  # a fake, 16-byte aligned "device" address; never dereferenced
+
+
+def _fwd(lib, q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
+    return lib.fattn_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, None)
+
+
+def test_fwd_validation(lib):
+    assert _fwd(lib, q=None) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, lse=None) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, B=0) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, H=-1) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, N=0) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, d=96) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, N=100) == binding.FATTN_ERR_UNSUPPORTED       # ragged length
+    assert _fwd(lib, B=1 << 14, H=1 << 10, N=1 << 8) == binding.FATTN_ERR_UNSUPPORTED  # 2^32 rows
+    assert _fwd(lib, scale=float("inf")) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, causal=2) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd(lib, k=P + 8) == binding.FATTN_ERR_ALIGNMENT
+    assert _fwd(lib, lse=P + 4) == binding.FATTN_ERR_ALIGNMENT
+
+
+def test_workspace_size(lib):
+    def a256(x):
+        return (x + 255) // 256 * 256
+    for (B, H, N, d) in [(1, 1, 128, 64), (4, 32, 4096, 128), (3, 5, 384, 128)]:
+        rows = B * H * N
+        assert lib.fattn_bwd_workspace_size(B, H, N, d) == 2 * a256(rows * 4) + a256(rows * d * 4)
+    assert lib.fattn_bwd_workspace_size(1, 1, 100, 64) == 0
+    assert lib.fattn_bwd_workspace_size(1, 1, 128, 96) == 0
+
+
+def _bwd(lib, ws=P, ws_bytes=None, d=64, N=128, **kw):
+    if ws_bytes is None:
+        ws_bytes = lib.fattn_bwd_workspace_size(1, 1, N, d) if d in (64, 128) and N % 128 == 0 else 1 << 30
+    args = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P)
+    args.update(kw)
+    return lib.fattn_bwd(args["q"], args["k"], args["v"], args["o"], args["do"], args["lse"], args["dq"],
+                         args["dk"], args["dv"], 1, 1, N, d, 0, 0.125, ws, ws_bytes, None)
+
+
+def test_bwd_validation(lib):
+    assert _bwd(lib, do=None) == binding.FATTN_ERR_INVALID_ARG
+    assert _bwd(lib, ws=None) == binding.FATTN_ERR_INVALID_ARG
+    assert _bwd(lib, ws_bytes=16) == binding.FATTN_ERR_INVALID_ARG
+    assert _bwd(lib, d=32) == binding.FATTN_ERR_UNSUPPORTED
+    assert _bwd(lib, N=200) == binding.FATTN_ERR_UNSUPPORTED
+    assert _bwd(lib, dq=P + 2) == binding.FATTN_ERR_ALIGNMENT
+    assert _bwd(lib, ws=P + 16) == binding.FATTN_ERR_ALIGNMENT  # workspace wants 256 bytes
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.fwd(q, q, q)
