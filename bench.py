@@ -1,0 +1,419 @@
+"""Throughput of the fused exact-attention hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl fattn|reference]
+
+One step = one pass of the whole hot path over one batch: fattn_fwd (O, LSE)
+followed by the three backward stages (preprocess, dK/dV with dQ atomics, dQ
+convert).  The default workload is the d=128 causal training shape
+B=4, H=32, N=4096.  Every input tensor (256 MiB each) is larger than the 126 MB
+L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): each rank runs the same step on its own batch drawn with
+seed + rank (independent problems, no collective on the data path: weak
+scaling); the time is the max over ranks of the device-timed region.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on the
+host cores, one (batch, head) slice per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "attention fwd+bwd TFLOPS (bf16)"
+
+
+def load_peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), \
+            float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 1400.0, FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.15)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample(w, heads, seed_offset=0, budget_s=None):
+    """Time the fp64 oracle (forward + backward) on whole (batch, head) slices.
+
+    Returns (seconds, algorithmic FLOPs covered, heads done, cores, blas threads)."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_108_b200.workloads import make_inputs, to_f64
+
+    q, k, v, do = make_inputs(w.B, w.H, w.N, w.d, w.seed + seed_offset, w.dist, True)
+    per_head = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.H)
+    t_total, done = 0.0, 0
+    for idx in heads:
+        b, h = divmod(idx, w.H)
+        qh, kh, vh, doh = (to_f64(t[b, h]) for t in (q, k, v, do))
+        t0 = time.perf_counter()
+        o, lse = oracle.ref_fwd(qh[None, None], kh[None, None], vh[None, None], w.causal, w.scale)
+        grads = oracle.ref_bwd_head(qh, kh, vh, doh, w.causal, w.scale)
+        t_total += time.perf_counter() - t0
+        done += 1
+        assert np.isfinite(o).all() and all(np.isfinite(g).all() for g in grads)
+        if budget_s is not None and t_total >= budget_s:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"),
+                   default=1)
+    except Exception:
+        blas = None
+    cores = len(os.sched_getaffinity(0))
+    return t_total, per_head * done, done, cores, blas
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from exact_attention_108_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    nheads = w.B * w.H
+    # each step = one (batch, head) slice, fwd + bwd; cap the whole run near 3 minutes
+    t_warm, _, _, cores, blas = oracle_sample(w, [0])
+    per_step = max(t_warm, 1e-3)
+    total_steps = args.steps + args.warmup
+    cap = max(2, int(180.0 / per_step))
+    steps = min(args.steps, max(1, cap - min(args.warmup, 1)))
+    warm = min(args.warmup, max(0, cap - steps))
+    heads = [(i * 7919) % nheads for i in range(1, warm + steps + 1)]
+    if warm > 1:
+        oracle_sample(w, heads[:warm - 1])
+    t, flops, done, cores, blas = oracle_sample(w, heads[warm:warm + steps])
+    tflops = flops / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOPS", "n_gpus": world,
+        "steps": done, "warmup": warm, "ms_per_step": 1e3 * t / done, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "reference": "fp64 CPU oracle (oracle/attention_fp64.py), one (batch, head) slice per step"},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOPS", "cores": cores, "blas_threads": blas,
+                         "kind": "oracle",
+                         "sample": f"{done} of {nheads} (batch, head) slices, fwd+bwd, full N={w.N}"},
+        "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "requested_steps": args.steps, "requested_warmup": args.warmup, "note": f"{total_steps} requested",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ multi-rank
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling, no data exchange)."""
+    return base_seed + rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank device-timed quantity (every rank calls this in the same order)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
+def dominant_kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed after the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for name in rec.get("sources", []):
+        try:
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    entry = rec.get("kernels", {}).get(kernel, {}).get(workload)
+    if not entry or entry.get("sources_sha256") != h.hexdigest():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def gpu_smi_id(torch, dev):
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return "%04x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return str(dev.index or 0)
+
+
+# ------------------------------------------------------------- GPU arm
+def run_fattn(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_108_b200 import binding
+    from exact_attention_108_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    if not w.backward:
+        raise SystemExit(f"workload {w.name} is forward-only; the bench step is forward + backward")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    binding.load()
+
+    q_h, k_h, v_h, do_h = make_inputs(w.B, w.H, w.N, w.d, rank_seed(w.seed, rank), w.dist, True)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(binding.workspace_size(w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 4  # fwd, bwd preprocess, bwd dK/dV, bwd dQ convert
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        binding.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        binding.bwd_preprocess(o, lse, do, ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        binding.bwd_dkdv(q, k, v, do, dk, dv, ws, causal=w.causal, scale=w.scale, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        binding.bwd_dq(dq, ws, scale=w.scale, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if binding.device_status(clear=True) != 0:
+        raise SystemExit("kernel wait timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_smi_id(torch, dev))
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier()
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    status = binding.device_status(clear=True)
+
+    stage = [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(4)]
+    fwd_ms = statistics.mean(stage[0])
+    pre_ms, dkdv_ms, dqc_ms = (statistics.mean(s) for s in stage[1:])
+    bwd_ms = pre_ms + dkdv_ms + dqc_ms
+    step_flops = w.fwd_flops() + w.bwd_flops()
+    ms_per_step = elapsed_ms / args.steps
+    value = whole_job_tflops(world, step_flops, ms_per_step)
+
+    peak, peak_sus, hbm, peak_kind = load_peaks()
+    dkdv_tflops = w.bwd_flops() / (dkdv_ms * 1e-3) / 1e12
+    fwd_tflops = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+    bwd_tflops = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
+        outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (q_h, k_h, v_h)]
+        e_steps = max(1, min(args.steps, args.e2e_steps))
+        for rep in range(2):  # first pass warms the copy engines
+            barrier()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(e_steps if rep else 1):
+                for dst, src in zip((q, k, v, do), pin):
+                    dst.copy_(src, non_blocking=True)
+                binding.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+                binding.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                            workspace=ws, stream=stream)
+                for dst, src in zip(outs, (dq, dk, dv)):
+                    dst.copy_(src, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+        e2e = {"value": whole_job_tflops(world, step_flops, e_ms), "unit": "TFLOPS",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs),
+               "ms_per_step": e_ms, "steps": e_steps,
+               "path": "pinned host Q,K,V,dO -> device; fattn_fwd; fattn_bwd; dQ,dK,dV -> pinned host"}
+
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        nheads = w.B * w.H
+        sample_heads = [0, nheads - 1] + [(i * 7919) % nheads for i in range(1, 30)]
+        t, flops, done, cores, blas = oracle_sample(w, sample_heads, budget_s=args.cpu_budget_s)
+        cpu = {"value": flops / t / 1e12, "unit": "TFLOPS", "cores": cores, "blas_threads": blas,
+               "kind": "oracle", "seconds": round(t, 2),
+               "sample": f"{done} of {w.B * w.H} (batch, head) slices of {w.name}, fwd+bwd at full N={w.N}, "
+                         f"scaled by FLOPs"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "dist": w.dist, "global_batch": w.B * world,
+                   "l2": "inputs larger than L2 (each of Q,K,V,dO,O is "
+                         f"{w.B * w.H * w.N * w.d * 2 / 2**20:.0f} MiB > 126 MB); no flush"},
+        "fwd_tflops": round(fwd_tflops, 1), "bwd_tflops": round(bwd_tflops, 1),
+        "fwd_frac_of_peak": round(fwd_tflops / peak, 4), "bwd_frac_of_peak": round(bwd_tflops / peak, 4),
+        "stage_ms": {"fwd": round(fwd_ms, 4), "bwd_preprocess": round(pre_ms, 4),
+                     "bwd_dkdv": round(dkdv_ms, 4), "bwd_dq": round(dqc_ms, 4)},
+        "roofline": {"kernel": "fattn_bwd_dkdv_kernel", "bound": "tensor", "achieved": round(dkdv_tflops, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(dkdv_tflops / peak, 4),
+                     "peak_kind": f"{peak_kind} bf16 burst (cuBLAS); sustained {peak_sus}",
+                     "algorithmic": "2.5 x 4*B*H*N^2*d (halved when causal) per launch",
+                     "traffic": args.traffic_bytes if args.traffic_bytes is not None
+                     else dominant_kernel_traffic("fattn_bwd_dkdv_kernel", w.name)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("fattn", "reference"), default="fattn")
+    ap.add_argument("--workload", default="train_d128_causal")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "fattn":
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_fattn(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -23,8 +23,9 @@ FATTN_ERR_CUDA = 4
 FATTN_ERR_DEVICE_TIMEOUT = 5
 
 # Every symbol include/fattn.h declares (checked by the CPU test suite).
-EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_status_string",
-            "fattn_last_cuda_error", "fattn_device_status", "fattn_version")
+EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_bwd_preprocess",
+            "fattn_bwd_dkdv", "fattn_bwd_dq", "fattn_status_string", "fattn_last_cuda_error",
+            "fattn_device_status", "fattn_version")
 
 _lib = None
 
@@ -51,6 +52,12 @@ def load():
     L.fattn_fwd.restype = i
     L.fattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     L.fattn_bwd.restype = i
+    L.fattn_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+    L.fattn_bwd_preprocess.restype = i
+    L.fattn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+    L.fattn_bwd_dkdv.restype = i
+    L.fattn_bwd_dq.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
+    L.fattn_bwd_dq.restype = i
     L.fattn_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fattn_bwd_workspace_size.restype = sz
     L.fattn_status_string.argtypes = [i]
@@ -148,3 +155,37 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
     if rc != FATTN_OK:
         raise FattnError(rc, "fattn_bwd")
     return dq, dk, dv
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def bwd_preprocess(o, lse, do, workspace, stream=None):
+    """Stage 1 of the backward: D, LSE*log2(e) and a zeroed dQ accumulator in `workspace`."""
+    B, H, N, d = _shape4(o)
+    rc = load().fattn_bwd_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d,
+                                     workspace.data_ptr(), _nbytes(workspace), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_bwd_preprocess")
+
+
+def bwd_dkdv(q, k, v, do, dk, dv, workspace, causal: bool = False, scale: float | None = None, stream=None):
+    """Stage 2: dK, dV, and dS K added into the workspace accumulator."""
+    B, H, N, d = _shape4(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rc = load().fattn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), B, H, N, d, 1 if causal else 0, float(scale),
+                               workspace.data_ptr(), _nbytes(workspace), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_bwd_dkdv")
+
+
+def bwd_dq(dq, workspace, scale: float | None = None, stream=None):
+    """Stage 3: dQ = bf16(scale * accumulator)."""
+    B, H, N, d = _shape4(dq)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    rc = load().fattn_bwd_dq(dq.data_ptr(), B, H, N, d, float(scale), workspace.data_ptr(),
+                             _nbytes(workspace), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_bwd_dq")

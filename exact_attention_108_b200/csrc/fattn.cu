@@ -122,34 +122,46 @@ int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   return FATTN_OK;
 }
 
-template <int D>
-int launch_bwd_d(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                 void* dq, void* dk, void* dv, int B, int H, int N, int causal, float scale, void* workspace,
-                 cudaStream_t st) {
-  const long long rows = (long long)B * H * N;
-  char* ws = static_cast<char*>(workspace);
-  float* dvec = reinterpret_cast<float*>(ws);
-  float* lse2 = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
-  float* dq_acc = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+struct WsParts {
+  float* dvec;
+  float* lse2;
+  float* dq_acc;
+};
 
-  {
-    constexpr int rpb = 256 / (D / 8);
-    const long long blocks = (rows + rpb - 1) / rpb;
-    fattn::fattn_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dq_acc,
-        rows);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_pre_kernel launch");
-  }
+WsParts split_workspace(void* workspace, long long rows) {
+  char* ws = static_cast<char*>(workspace);
+  WsParts p;
+  p.dvec = reinterpret_cast<float*>(ws);
+  p.lse2 = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
+  p.dq_acc = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+  return p;
+}
+
+template <int D>
+int launch_pre(const void* o, const void* dout, const float* lse, long long rows, const WsParts& w, cudaStream_t st) {
+  constexpr int rpb = 256 / (D / 8);
+  const long long blocks = (rows + rpb - 1) / rpb;
+  fattn::fattn_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                                    static_cast<const __nv_bfloat16*>(dout), lse,
+                                                                    w.dvec, w.lse2, w.dq_acc, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_pre_kernel launch");
+  return FATTN_OK;
+}
+
+template <int D>
+int launch_dkdv_d(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
+                  int N, int causal, float scale, const WsParts& w, cudaStream_t st) {
+  const long long rows = (long long)B * H * N;
   CUtensorMap mq, mk, mv, mdo;
   if (int rc = make_bf16_tile_map(&mq, q, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mk, k, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mv, v, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mdo, dout, rows, D)) return rc;
   fattn::BwdArgs a;
-  a.lse2 = lse2;
-  a.dvec = dvec;
-  a.dq_acc = dq_acc;
+  a.lse2 = w.lse2;
+  a.dvec = w.dvec;
+  a.dq_acc = w.dq_acc;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.N = N;
@@ -157,18 +169,33 @@ int launch_bwd_d(const void* q, const void* k, const void* v, const void* o, con
   a.scale = scale;
   a.scale_log2 = scale * kLog2e;
   const int BH = B * H;
-  int rc = causal ? launch_dkdv<D, true>(mq, mk, mv, mdo, a, BH, st) : launch_dkdv<D, false>(mq, mk, mv, mdo, a, BH, st);
-  if (rc) return rc;
-  {
-    const long long n8 = rows * D / 8;
-    long long blocks = (n8 + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    fattn::fattn_bwd_dq_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), scale,
-                                                                     n8);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dq_kernel launch");
-  }
+  return causal ? launch_dkdv<D, true>(mq, mk, mv, mdo, a, BH, st) : launch_dkdv<D, false>(mq, mk, mv, mdo, a, BH, st);
+}
+
+template <int D>
+int launch_dq(void* dq, long long rows, float scale, const WsParts& w, cudaStream_t st) {
+  const long long n8 = rows * D / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  fattn::fattn_bwd_dq_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), scale, n8);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dq_kernel launch");
   return FATTN_OK;
+}
+
+int check_workspace(void* workspace, size_t bytes, int B, int H, int N, int d) {
+  if (!workspace) return FATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FATTN_ERR_ALIGNMENT;
+  const long long rows = (long long)B * H * N;
+  const size_t need = 2 * align256(rows * sizeof(float)) + align256(rows * (size_t)d * sizeof(float));
+  if (bytes < need) return FATTN_ERR_INVALID_ARG;
+  return FATTN_OK;
+}
+
+int check_common(int B, int H, int N, int d, float scale, int causal) {
+  if (!std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FATTN_ERR_INVALID_ARG;
+  return check_shape(B, H, N, d);
 }
 
 }  // namespace
@@ -238,20 +265,57 @@ size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {
   return 2 * align256(rows * sizeof(float)) + align256(rows * (size_t)d * sizeof(float));
 }
 
+int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, fattn_stream_t stream) {
+  if (!o || !dout || !lse || !workspace) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_common(B, H, N, d, 1.f, 0)) return rc;
+  if (!aligned16(o) || !aligned16(dout) || !aligned16(lse)) return FATTN_ERR_ALIGNMENT;
+  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
+  const long long rows = (long long)B * H * N;
+  const WsParts w = split_workspace(workspace, rows);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_pre<64>(o, dout, lse, rows, w, st) : launch_pre<128>(o, dout, lse, rows, w, st);
+}
+
+int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
+                   int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                   fattn_stream_t stream) {
+  if (!q || !k || !v || !dout || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_common(B, H, N, d, scale, causal)) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
+    return FATTN_ERR_ALIGNMENT;
+  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
+  const WsParts w = split_workspace(workspace, (long long)B * H * N);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_dkdv_d<64>(q, k, v, dout, dk, dv, B, H, N, causal, scale, w, st)
+                 : launch_dkdv_d<128>(q, k, v, dout, dk, dv, B, H, N, causal, scale, w, st);
+}
+
+int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
+                 fattn_stream_t stream) {
+  if (!dq || !workspace) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_common(B, H, N, d, scale, 0)) return rc;
+  if (!aligned16(dq)) return FATTN_ERR_ALIGNMENT;
+  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
+  const long long rows = (long long)B * H * N;
+  const WsParts w = split_workspace(workspace, rows);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_dq<64>(dq, rows, scale, w, st) : launch_dq<128>(dq, rows, scale, w, st);
+}
+
 int fattn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
               void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
               size_t workspace_bytes, fattn_stream_t stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_shape(B, H, N, d)) return rc;
+  if (int rc = check_common(B, H, N, d, scale, causal)) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FATTN_ERR_ALIGNMENT;
-  if (workspace_bytes < fattn_bwd_workspace_size(B, H, N, d)) return FATTN_ERR_INVALID_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) return launch_bwd_d<64>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, workspace, st);
-  return launch_bwd_d<128>(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, causal, scale, workspace, st);
+  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
+  if (int rc = fattn_bwd_preprocess(o, dout, lse, B, H, N, d, workspace, workspace_bytes, stream)) return rc;
+  if (int rc = fattn_bwd_dkdv(q, k, v, dout, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes, stream))
+    return rc;
+  return fattn_bwd_dq(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

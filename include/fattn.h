@@ -93,6 +93,27 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o,
               int B, int H, int N, int d, int causal, float scale,
               void* workspace, size_t workspace_bytes, fattn_stream_t stream);
 
+/*
+ * The three stages fattn_bwd runs, exposed so that callers can schedule or time
+ * them separately.  They must run in this order on one stream with the same
+ * shape, scale and workspace; fattn_bwd(...) is exactly
+ *   fattn_bwd_preprocess; fattn_bwd_dkdv; fattn_bwd_dq.
+ *
+ * fattn_bwd_preprocess: D_i = sum_c dout_ic o_ic and LSE_i*log2(e) into the
+ *   workspace, and zeroes the workspace's fp32 dQ accumulator.
+ * fattn_bwd_dkdv: writes dk, dv and adds dS K (unscaled) into the accumulator.
+ *   Reads q, k, v, dout and the preprocess results.
+ * fattn_bwd_dq: dq = bf16(scale * accumulator).
+ * Validation and errors are those of fattn_bwd.
+ */
+int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, fattn_stream_t stream);
+int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                   int B, int H, int N, int d, int causal, float scale,
+                   void* workspace, size_t workspace_bytes, fattn_stream_t stream);
+int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale,
+                 void* workspace, size_t workspace_bytes, fattn_stream_t stream);
+
 /* Static, human-readable text for a status code. */
 const char* fattn_status_string(int status);
 

@@ -1,0 +1,123 @@
+"""Full-size GPU parity on the five workloads, in the launch configuration bench.py
+times (fattn_fwd then the three backward stages).
+
+At full size the oracle runs on what it can compute one by one:
+* whole (batch, head) slices (fwd + bwd) for two labelled heads per workload;
+* sampled query rows of O, LSE and dQ on every head (each needs only its own row);
+and properties that hold at any size check the rest on every head:
+* Q = 0 gives uniform (prefix-mean) attention, exactly representable on the GPU;
+* sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i per head.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_108_b200 import binding
+from exact_attention_108_b200.workloads import WORKLOADS, to_f64
+from gpu_common import assert_device_ok, check_grad, check_lse, check_o, gpu_inputs
+
+pytestmark = pytest.mark.gpu
+
+ROWS_PER_HEAD = 6
+
+
+def _run(w):
+    cpu, (q, k, v, do) = gpu_inputs(w.B, w.H, w.N, w.d, w.seed, w.dist, with_do=w.backward)
+    o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    grads = None
+    if w.backward:
+        ws = torch.empty(binding.workspace_size(w.B, w.H, w.N, w.d), device=q.device, dtype=torch.uint8)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        binding.bwd_preprocess(o, lse, do, ws)
+        binding.bwd_dkdv(q, k, v, do, dk, dv, ws, causal=w.causal, scale=w.scale)
+        binding.bwd_dq(dq, ws, scale=w.scale)
+        grads = (dq, dk, dv)
+    assert_device_ok()
+    return cpu, (q, k, v, do), o, lse, grads
+
+
+def _sampled_rows(N, rng):
+    rows = {0, 1, 127, 128, N - 1}
+    rows.update(rng.integers(0, N, ROWS_PER_HEAD).tolist())
+    return sorted(rows)
+
+
+def _check_workload(w, full_heads):
+    cpu, gpu, o, lse, grads = _run(w)
+    q, k, v, do = cpu
+    rng = np.random.default_rng(w.seed)
+    # every head: sampled rows of O, LSE (and dQ)
+    for b in range(w.B):
+        for h in range(w.H):
+            rows = _sampled_rows(w.N, rng)
+            qh, kh, vh = (to_f64(t[b, h]) for t in (q, k, v))
+            o_r, l_r = oracle.ref_fwd_rows(qh, kh, vh, rows, w.causal, w.scale)
+            check_o(to_f64(o[b, h, rows]), o_r, f"head ({b},{h}) rows")
+            check_lse(lse[b, h, rows], l_r, f"head ({b},{h}) rows")
+            if grads is not None:
+                doh = to_f64(do[b, h])
+                dq_r = oracle.ref_dq_rows(qh, kh, vh, doh, rows, w.causal, w.scale)
+                err = np.abs(to_f64(grads[0][b, h, rows]) - dq_r).max()
+                # row samples: bound by the head's largest sampled reference magnitude
+                assert err <= 2e-2 * np.abs(dq_r).max() + 1e-6, f"dQ rows head ({b},{h}): {err}"
+    # labelled heads: everything
+    for (b, h) in full_heads:
+        qh, kh, vh = (to_f64(t[b, h]) for t in (q, k, v))
+        o_ref, lse_ref = oracle.ref_fwd(qh[None, None], kh[None, None], vh[None, None], w.causal, w.scale)
+        check_o(to_f64(o[b, h]), o_ref[0, 0], f"head ({b},{h})")
+        check_lse(lse[b, h], lse_ref[0, 0], f"head ({b},{h})")
+        if grads is not None:
+            doh = to_f64(do[b, h])
+            refs = oracle.ref_bwd_head(qh, kh, vh, doh, w.causal, w.scale)
+            for g, r, n in zip(grads, refs, ("dQ", "dK", "dV")):
+                check_grad(to_f64(g[b, h]), r, n, f"head ({b},{h})")
+    # every head: column-sum invariants of the backward.  bf16 rounding of the
+    # individual rows makes the sums inexact, so they are bounded relative to the
+    # sum of magnitudes (a gross error -- a dropped term, a wrong mask -- breaks this).
+    if grads is not None:
+        dq, dk, dv = grads
+        dkd, dvd, dod = dk.double(), dv.double(), do.double()
+        rel_k = dkd.sum(dim=2).abs() / dkd.abs().sum(dim=2).clamp_min(1e-30)
+        assert rel_k.max().item() <= 1e-2, f"sum_j dK_j != 0 (rel {rel_k.max().item():.2e})"
+        rel_v = (dvd.sum(dim=2) - dod.sum(dim=2)).abs() / dvd.abs().sum(dim=2).clamp_min(1e-30)
+        assert rel_v.max().item() <= 1e-2, f"sum_j dV_j != sum_i dO_i (rel {rel_v.max().item():.2e})"
+
+
+def test_fwd_d64_full_size():
+    _check_workload(WORKLOADS["fwd_d64"], [(0, 0), (7, 15)])
+
+
+def test_fwd_d64_causal_full_size():
+    _check_workload(WORKLOADS["fwd_d64_causal"], [(0, 0), (7, 15)])
+
+
+def test_train_d128_causal_full_size():
+    _check_workload(WORKLOADS["train_d128_causal"], [(0, 0), (3, 31)])
+
+
+def test_peaked_n8192_full_size():
+    _check_workload(WORKLOADS["peaked_n8192"], [(0, 0), (1, 15)])
+
+
+@pytest.mark.slow
+def test_long_n32768_causal_full_size():
+    _check_workload(WORKLOADS["long_n32768_causal"], [(0, 0), (0, 7)])
+
+
+@pytest.mark.parametrize("name", ["train_d128_causal", "long_n32768_causal", "fwd_d64"])
+def test_zero_queries_closed_form_full_size(name):
+    """Q = 0: every weight is exp(0) = 1, so O is the (prefix) mean of V and LSE
+    = ln(count) on every head, at full size."""
+    w = WORKLOADS[name]
+    _, (q, k, v, _) = gpu_inputs(w.B, w.H, w.N, w.d, w.seed, w.dist, with_do=False)
+    q.zero_()
+    o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    assert_device_ok()
+    counts = torch.arange(1, w.N + 1, device=v.device, dtype=torch.float64) if w.causal else \
+        torch.full((w.N,), float(w.N), device=v.device, dtype=torch.float64)
+    vd = v.double()
+    mean = (vd.cumsum(dim=2) if w.causal else vd.sum(dim=2, keepdim=True).expand_as(vd)) / counts[:, None]
+    err = (o.double() - mean).abs()
+    assert err.max().item() <= 1e-2 and err.mean().item() <= 1e-3
+    assert (lse.double() - counts.log()).abs().max().item() <= 1e-3
