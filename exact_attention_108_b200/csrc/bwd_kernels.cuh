@@ -149,8 +149,12 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int NT = args.num_tiles;
-  const int kv_tile = (int)blockIdx.y;  // causal: small tiles see the most queries -> launched first
-  const int head_row0 = (int)blockIdx.x * args.N;
+  // The key tile varies fastest so that the CTAs resident at one time add into
+  // the same head's dQ rows (which then stay in L2); causal: tile 0 sees the most
+  // query tiles and is launched first.
+  const int bh = (int)(blockIdx.x / (unsigned)NT);
+  const int kv_tile = (int)(blockIdx.x % (unsigned)NT);
+  const int head_row0 = bh * args.N;
   const int kv_row0 = head_row0 + kv_tile * 128;
   const int i_begin = CAUSAL ? kv_tile : 0;
   const int n_q = NT - i_begin;

@@ -81,7 +81,7 @@ int check_shape(int B, int H, int N, int d) {
   if (N % 128 != 0) return FATTN_ERR_UNSUPPORTED;
   const long long rows = (long long)B * H * N;
   if (rows >= (1ll << 31)) return FATTN_ERR_UNSUPPORTED;
-  if ((long long)H * B > 0x7fffffffll || N / 128 > 65535) return FATTN_ERR_UNSUPPORTED;
+  if (rows / 128 > 0x7fffffffll) return FATTN_ERR_UNSUPPORTED;  // one CTA per 128-row tile
   return FATTN_OK;
 }
 
@@ -98,7 +98,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   auto kern = fattn::fattn_fwd_kernel<D, CAUSAL>;
   constexpr int smem = fattn::FwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
-  dim3 grid((unsigned)BH, (unsigned)a.num_q_tiles);
+  dim3 grid((unsigned)((long long)BH * a.num_q_tiles));
   kern<<<grid, 256, smem, st>>>(mq, mk, mv, mo, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_fwd_kernel launch");
@@ -115,7 +115,7 @@ int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   auto kern = fattn::fattn_bwd_dkdv_kernel<D, CAUSAL>;
   constexpr int smem = fattn::BwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
-  dim3 grid((unsigned)BH, (unsigned)a.num_tiles);
+  dim3 grid((unsigned)((long long)BH * a.num_tiles));
   kern<<<grid, 256, smem, st>>>(mq, mk, mv, mdo, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dkdv_kernel launch");

@@ -92,10 +92,13 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: blockIdx.x = batch*head, blockIdx.y = query tile (longest first when causal).
+  // Work unit: the query tile varies fastest so that the CTAs resident at one
+  // time share a head's K/V in L2; causal heads run their longest tiles first.
   const int NT = args.num_q_tiles;
-  const int q_tile = CAUSAL ? (NT - 1 - (int)blockIdx.y) : (int)blockIdx.y;
-  const int head_row0 = (int)blockIdx.x * args.N;
+  const int bh = (int)(blockIdx.x / (unsigned)NT);
+  const int t_in_head = (int)(blockIdx.x % (unsigned)NT);
+  const int q_tile = CAUSAL ? (NT - 1 - t_in_head) : t_in_head;
+  const int head_row0 = bh * args.N;
   const int q_row0 = head_row0 + q_tile * C::BM;
   const int n_kv = CAUSAL ? (q_tile + 1) : NT;
 
