@@ -7,14 +7,16 @@
 //  1. fattn_bwd_pre_kernel   D_i = sum_c dO_ic O_ic, LSE2_i = LSE_i log2(e),
 //                            and zero the fp32 dQ accumulator.     (HBM-bound)
 //  2. fattn_bwd_dkdv_kernel  one CTA per (batch*head, 128-row key tile j);
-//                            loops over the 128-row query tiles i that can see
-//                            tile j and, on the tcgen05 tensor cores,
-//                              S^T  = K_j Q_i^T          (TMEM)
+//                            loops over the 64-row query sub-tiles i that can
+//                            see tile j and, on the tcgen05 tensor cores,
+//                              S^T  = K_j Q_i^T          (TMEM, two buffers)
 //                              dP^T = V_j dO_i^T         (TMEM)
 //                              P^T  = exp2(S^T scale log2e - LSE2_i)   (masked)
 //                              dS^T = P^T o (dP^T - D_i)
-//                              dV_j += P^T dO_i,  dK_j += dS^T Q_i  (TMEM accumulators)
-//                              dQ_i += dS K_j  -> fp32 atomics into the accumulator
+//                              dV_j += P^T dO_i   (P^T read from TMEM)
+//                              dK_j += dS^T Q_i   (TMEM accumulators)
+//                              dQ_i^T = K_j^T dS^T_i -> fp32 atomics into the
+//                                                       accumulator
 //                            (atomic global updates, page 3 "5.3 专用指令利用").
 //  3. fattn_bwd_dq_kernel    dQ = bf16(scale * accumulator).
 #pragma once
@@ -80,69 +82,87 @@ __global__ void __launch_bounds__(256) fattn_bwd_dq_kernel(const float* __restri
 
 // ------------------------------------------------------------------ kernel 2
 struct BwdArgs {
-  const float* lse2;   // [B*H*N]  LSE * log2(e)
-  const float* dvec;   // [B*H*N]  D
-  float* dq_acc;       // [B*H*N, D] fp32
-  __nv_bfloat16* dk;   // [B*H*N, D]
-  __nv_bfloat16* dv;   // [B*H*N, D]
+  const float* lse2;  // [B*H*N]  LSE * log2(e)
+  const float* dvec;  // [B*H*N]  D
+  float* dq_acc;      // [B*H*N, D] fp32
   int N;
-  int num_tiles;       // N / 128
-  float scale;         // for dK
-  float scale_log2;    // scale * log2(e)
+  int num_tiles;      // N / 128
+  float scale;        // for dK
+  float scale_log2;   // scale * log2(e)
 };
 
 template <int D>
 struct BwdCfg {
-  static constexpr int KB = D / 64;
-  static constexpr int TILE = 128 * D * 2;
+  static constexpr int KB = D / 64;              // 64-column (128-byte) blocks per row
+  static constexpr int BQ = 64;                  // query rows per inner step
+  static constexpr int NS = 3;                   // Q/dO ring depth
+  static constexpr int KV_TILE = 128 * D * 2;    // bytes of the K (or V) tile
+  static constexpr int KV_BLK = 128 * 128;       // one 64-column block of a 128-row tile
+  static constexpr int Q_TILE = BQ * D * 2;      // bytes of a Q (or dO) sub-tile
+  static constexpr int Q_BLK = BQ * 128;         // one 64-column block of a 64-row sub-tile
+  static constexpr int DS_BYTES = 128 * BQ * 2;  // dS^T [128 keys][64 queries] bf16
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = TILE;
-  static constexpr int OFF_Q = 2 * TILE;
-  static constexpr int OFF_DO = 3 * TILE;
-  static constexpr int OFF_PT = 4 * TILE;                 // P^T  [128 kv][128 q] bf16, 32 KB
-  static constexpr int OFF_DST = OFF_PT + 32768;          // dS^T [128 kv][128 q] bf16, 32 KB
-  static constexpr int OFF_LSE = OFF_DST + 32768;         // 128 fp32
-  static constexpr int OFF_DV = OFF_LSE + 512;            // 128 fp32
-  static constexpr int OFF_BAR = OFF_DV + 512;
-  // kv_full, qdo_full, qdo_empty, st_full, ds_full, dq_full, tm_free, done, drain
-  static constexpr int NBAR = 9;
+  static constexpr int OFF_V = KV_TILE;
+  static constexpr int OFF_STAGE = 2 * KV_TILE;
+  static constexpr int STAGE = 2 * Q_TILE;       // Q sub-tile, then dO sub-tile
+  static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
+  static constexpr int OFF_STAT = OFF_DS + 2 * DS_BYTES;  // per stage: LSE2[64], D[64] fp32
+  static constexpr int OFF_BAR = OFF_STAT + NS * 512;
+  // kv_full, q_full[NS], q_empty[NS], st_full[2], ds_full[2], pv_done[2], dq_full, dq_free, done, drain
+  static constexpr int NBAR = 1 + 2 * NS + 6 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 256 + D, TM_DQ = 128;
+  // S^T buffers (P^T as bf16 overlays their first 32 columns), dP^T, dQ^T, dV, dK
+  static constexpr int TM_S0 = 0, TM_S1 = 64, TM_DP = 128, TM_DQ = 192, TM_DV = 256, TM_DK = 256 + D;
 };
 
 enum : int {
   kSiteBwdProducer = 0x201,
   kSiteBwdMmaKV = 0x202,
   kSiteBwdMmaQ = 0x203,
-  kSiteBwdMmaFree = 0x204,
+  kSiteBwdMmaPV = 0x204,
   kSiteBwdMmaDS = 0x205,
-  kSiteBwdSoftS = 0x206,
-  kSiteBwdSoftQ = 0x207,
-  kSiteBwdSoftDQ = 0x208,
-  kSiteBwdEpi = 0x209,
+  kSiteBwdMmaDQ = 0x206,
+  kSiteBwdSoftS = 0x207,
+  kSiteBwdSoftQ = 0x208,
+  kSiteBwdDrain = 0x209,
+  kSiteBwdEpi = 0x20a,
 };
 
+// Roles (320 threads):
+//   warps 0..3  softmax-gradient group, thread = key row of the tile: P^T, dS^T
+//   warps 4..7  dQ drain (thread = head-dim lane of dQ^T) and the dK/dV epilogue
+//   warp 8      TMA producer (K, V once; Q/dO sub-tiles through an NS-deep ring)
+//   warp 9      tcgen05 issuer (one thread)
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(320, 1)
     fattn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                           const BwdArgs args) {
   using C = BwdCfg<D>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
-  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sQ = sbase + C::OFF_Q, sDO = sbase + C::OFF_DO;
-  const uint32_t sPT = sbase + C::OFF_PT, sDST = sbase + C::OFF_DST;
-  const uint32_t sLSE = sbase + C::OFF_LSE, sDvec = sbase + C::OFF_DV;
-  const float* lse_s = reinterpret_cast<const float*>(smem + C::OFF_LSE);
-  const float* dvec_s = reinterpret_cast<const float*>(smem + C::OFF_DV);
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
+  auto sQ = [&](int s) { return sbase + C::OFF_STAGE + s * C::STAGE; };
+  auto sDO = [&](int s) { return sbase + C::OFF_STAGE + s * C::STAGE + C::Q_TILE; };
+  auto sDS = [&](int b) { return sbase + C::OFF_DS + b * C::DS_BYTES; };
+  auto sStat = [&](int s) { return sbase + C::OFF_STAT + s * 512; };
+  auto stat = [&](int s) { return reinterpret_cast<const float*>(smem + C::OFF_STAT + s * 512); };
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t bar_kv_full = bar0, bar_qdo_full = bar0 + 8, bar_qdo_empty = bar0 + 16;
-  const uint32_t bar_st_full = bar0 + 24, bar_ds_full = bar0 + 32, bar_dq_full = bar0 + 40;
-  const uint32_t bar_tm_free = bar0 + 48, bar_done = bar0 + 56, bar_drain = bar0 + 64;
+  const uint32_t bar_kv_full = bar0;
+  auto bar_q_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_q_empty = [&](int s) { return bar0 + 8u * (1 + C::NS + s); };
+  auto bar_st_full = [&](int b) { return bar0 + 8u * (1 + 2 * C::NS + b); };
+  auto bar_ds_full = [&](int b) { return bar0 + 8u * (3 + 2 * C::NS + b); };
+  auto bar_pv_done = [&](int b) { return bar0 + 8u * (5 + 2 * C::NS + b); };
+  const uint32_t bar_dq_full = bar0 + 8u * (7 + 2 * C::NS);
+  const uint32_t bar_dq_free = bar0 + 8u * (8 + 2 * C::NS);
+  const uint32_t bar_done = bar0 + 8u * (9 + 2 * C::NS);
+  const uint32_t bar_drain = bar0 + 8u * (10 + 2 * C::NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -151,28 +171,33 @@ __global__ void __launch_bounds__(256, 1)
   const int NT = args.num_tiles;
   // The key tile varies fastest so that the CTAs resident at one time add into
   // the same head's dQ rows (which then stay in L2); causal: tile 0 sees the most
-  // query tiles and is launched first.
+  // query rows and is launched first.
   const int bh = (int)(blockIdx.x / (unsigned)NT);
   const int kv_tile = (int)(blockIdx.x % (unsigned)NT);
   const int head_row0 = bh * args.N;
   const int kv_row0 = head_row0 + kv_tile * 128;
-  const int i_begin = CAUSAL ? kv_tile : 0;
-  const int n_q = NT - i_begin;
+  const int q_begin = CAUSAL ? kv_tile * 128 : 0;  // first query row (in the head) that sees this tile
+  const int n_it = (args.N - q_begin) / C::BQ;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
-    mbar_init(bar_qdo_full, 1);
-    mbar_init(bar_qdo_empty, 1);
-    mbar_init(bar_st_full, 1);
-    mbar_init(bar_ds_full, 128);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar_q_full(s), 1);
+      mbar_init(bar_q_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_st_full(b), 1);
+      mbar_init(bar_ds_full(b), 128);
+      mbar_init(bar_pv_done(b), 1);
+    }
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_tm_free, 128);
+    mbar_init(bar_dq_free, 128);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -181,193 +206,228 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
       prefetch_tensormap(&tm_do);
-      mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
+      mbar_arrive_expect_tx(bar_kv_full, 2 * C::KV_TILE);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb) {
-        tma_load_2d(sK + kb * 16384, &tm_k, bar_kv_full, kb * 64, kv_row0);
-        tma_load_2d(sV + kb * 16384, &tm_v, bar_kv_full, kb * 64, kv_row0);
+        tma_load_2d(sK + kb * C::KV_BLK, &tm_k, bar_kv_full, kb * 64, kv_row0);
+        tma_load_2d(sV + kb * C::KV_BLK, &tm_v, bar_kv_full, kb * 64, kv_row0);
       }
       int it = 0;
-      for (; it < n_q; ++it) {
-        if (!mbar_wait(bar_qdo_empty, (it & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
-        const int q_row0 = head_row0 + (i_begin + it) * 128;
-        mbar_arrive_expect_tx(bar_qdo_full, 2 * C::TILE + 1024);
+      for (; it < n_it; ++it) {
+        const int s = it % C::NS;
+        if (!mbar_wait(bar_q_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
+        const int q_row = head_row0 + q_begin + it * C::BQ;
+        mbar_arrive_expect_tx(bar_q_full(s), C::STAGE + 512);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_2d(sQ + kb * 16384, &tm_q, bar_qdo_full, kb * 64, q_row0);
-          tma_load_2d(sDO + kb * 16384, &tm_do, bar_qdo_full, kb * 64, q_row0);
+          tma_load_2d(sQ(s) + kb * C::Q_BLK, &tm_q, bar_q_full(s), kb * 64, q_row);
+          tma_load_2d(sDO(s) + kb * C::Q_BLK, &tm_do, bar_q_full(s), kb * 64, q_row);
         }
-        bulk_load(sLSE, args.lse2 + q_row0, 512, bar_qdo_full);
-        bulk_load(sDvec, args.dvec + q_row0, 512, bar_qdo_full);
+        bulk_load(sStat(s), args.lse2 + q_row, 256, bar_q_full(s));
+        bulk_load(sStat(s) + 256, args.dvec + q_row, 256, bar_q_full(s));
       }
-      if (it < n_q) {  // aborted: let issued copies land
+      if (it < n_it) {  // aborted: let the copies already issued land
         mbar_wait_ns(bar_kv_full, 0, 100000000ull);
-        if (it > 0) mbar_wait_ns(bar_qdo_full, (it - 1) & 1, 100000000ull);
+        for (int i = (it > C::NS ? it - C::NS : 0); i < it; ++i)
+          mbar_wait_ns(bar_q_full(i % C::NS), (i / C::NS) & 1, 100000000ull);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // K/V (K-major) x Q/dO (K-major)
-      constexpr uint32_t id_kv = idesc_bf16_f32(128, D, false, true);    // P^T/dS^T (K-major) x dO/Q (MN-major)
-      constexpr uint32_t id_q = idesc_bf16_f32(128, D, true, true);      // dS (MN-major) x K (MN-major)
+      constexpr uint32_t id_s = idesc_bf16_f32(128, C::BQ, false, false);  // K/V (K-major) x Q/dO (K-major)
+      constexpr uint32_t id_kv = idesc_bf16_f32(128, D, false, true);      // P^T|dS^T (K-major) x dO|Q (MN)
+      constexpr uint32_t id_q = idesc_bf16_f32(128, C::BQ, true, true);    // K^T (MN) x dS^T (MN)
+      // For d = 64 the dQ^T product still uses M = 128: the second 64-row half of
+      // A repeats the first (LBO = 0) and its output lanes are ignored.
+      constexpr uint32_t kt_lbo = (D == 128) ? C::KV_BLK : 0;
       bool ok = mbar_wait(bar_kv_full, 0, abort_flag, kSiteBwdMmaKV);
-      for (int it = 0; it < n_q && ok; ++it) {
-        if (!(ok = mbar_wait(bar_qdo_full, it & 1, abort_flag, kSiteBwdMmaQ))) break;
-        if (!(ok = mbar_wait(bar_tm_free, (it & 1) ^ 1, abort_flag, kSiteBwdMmaFree))) break;
+      auto issue_s_dp = [&](int it) -> bool {
+        const int s = it % C::NS, b = it & 1;
+        if (!mbar_wait(bar_q_full(s), (it / C::NS) & 1, abort_flag, kSiteBwdMmaQ)) return false;
+        // P^T of iteration it-2 lives in this S buffer: its dV product must be done
+        if (it >= 2 && !mbar_wait(bar_pv_done(b), ((it >> 1) & 1) ^ 1, abort_flag, kSiteBwdMmaPV)) return false;
         tc_fence_after();
+        const uint32_t tS = tmem + (b ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_ST, sdesc_sw128(sK + koff, 16), sdesc_sw128(sQ + koff, 16), id_s, kk > 0);
+          const uint32_t ka = (kk >> 2) * C::KV_BLK + (kk & 3) * 32;
+          const uint32_t kb = (kk >> 2) * C::Q_BLK + (kk & 3) * 32;
+          mma_ss(tS, sdesc_sw128(sK + ka, 16), sdesc_sw128(sQ(s) + kb, 16), id_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DPT, sdesc_sw128(sV + koff, 16), sdesc_sw128(sDO + koff, 16), id_s, kk > 0);
+          const uint32_t ka = (kk >> 2) * C::KV_BLK + (kk & 3) * 32;
+          const uint32_t kb = (kk >> 2) * C::Q_BLK + (kk & 3) * 32;
+          mma_ss(tmem + C::TM_DP, sdesc_sw128(sV + ka, 16), sdesc_sw128(sDO(s) + kb, 16), id_s, kk > 0);
         }
-        mma_commit(bar_st_full);
-        if (!(ok = mbar_wait(bar_ds_full, it & 1, abort_flag, kSiteBwdMmaDS))) break;
+        mma_commit(bar_st_full(b));
+        return true;
+      };
+      if (ok) ok = issue_s_dp(0);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it % C::NS, b = it & 1;
+        if (!(ok = mbar_wait(bar_ds_full(b), (it >> 1) & 1, abort_flag, kSiteBwdMmaDS))) break;
+        tc_fence_after();
+        if (it + 1 < n_it && !(ok = issue_s_dp(it + 1))) break;
+        const uint32_t tP = tmem + (b ? C::TM_S1 : C::TM_S0);
+        // dV += P^T dO  (A = P^T from TMEM: 4 x 16 query columns, 8 TMEM columns each)
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          mma_ts(tmem + C::TM_DV, tP + kk * 8, sdesc_sw128(sDO(s) + kk * 2048, C::Q_BLK), id_kv,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_pv_done(b));
+        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          mma_ss(tmem + C::TM_DK, sdesc_sw128(sDS(b) + kk * 32, 16), sdesc_sw128(sQ(s) + kk * 2048, C::Q_BLK),
+                 id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_q_empty(s));
+        // dQ^T = K^T dS^T once the previous dQ^T has been drained
+        if (!(ok = mbar_wait(bar_dq_free, (it & 1) ^ 1, abort_flag, kSiteBwdMmaDQ))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DV, sdesc_sw128(sPT + aoff, 16), sdesc_sw128(sDO + kk * 2048, 16384), id_kv,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DK, sdesc_sw128(sDST + aoff, 16), sdesc_sw128(sQ + kk * 2048, 16384), id_kv,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K = 128 key rows
-          mma_ss(tmem + C::TM_DQ, sdesc_sw128(sDST + kk * 2048, 16384), sdesc_sw128(sK + kk * 2048, 16384), id_q,
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::TM_DQ, sdesc_sw128(sK + kk * 2048, kt_lbo), sdesc_sw128(sDS(b) + kk * 2048, 16), id_q,
                  kk > 0 ? 1u : 0u);
-        }
         mma_commit(bar_dq_full);
-        mma_commit(bar_qdo_empty);
       }
       if (ok) mma_commit(bar_done);
       mma_commit(bar_drain);
       mbar_wait_ns(bar_drain, 0, 100000000ull);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
     // ------------------------------------------------- softmax-gradient group
-    const int wq = warp - 4;
-    const int r = wq * 32 + lane;  // key row of the tile for S^T/dP^T; query row for dQ
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int r = warp * 32 + lane;  // key row inside the tile
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int kv_idx = kv_tile * 128 + r;
     const float sl2 = args.scale_log2;
-    bool ok = true;
-    for (int it = 0; it < n_q; ++it) {
-      const int i = i_begin + it;
-      ok = mbar_wait(bar_st_full, it & 1, abort_flag, kSiteBwdSoftS);
-      ok = ok && mbar_wait(bar_qdo_full, it & 1, abort_flag, kSiteBwdSoftQ);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % C::NS, b = it & 1;
+      bool ok = mbar_wait(bar_st_full(b), (it >> 1) & 1, abort_flag, kSiteBwdSoftS);
+      ok = ok && mbar_wait(bar_q_full(s), (it / C::NS) & 1, abort_flag, kSiteBwdSoftQ);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const bool diag = CAUSAL && (i == kv_tile);
+      const uint32_t tS = tmem + (b ? C::TM_S1 : C::TM_S0) + lane_off;
+      const float* lse_s = stat(s);
+      const float* dvec_s = stat(s) + 64;
+      const int q0 = q_begin + it * C::BQ;  // first query row (in the head) of this sub-tile
+      const bool diag = CAUSAL && (q0 < kv_tile * 128 + 128);
+      uint32_t pk[32];  // P^T row, packed bf16 pairs
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t sv[32], pv[32];
-        tmem_ld32(tmem + C::TM_ST + lane_off + c4 * 32, sv);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + h * 32, sv);
         tmem_ld_wait(sv);
-        tmem_ld32(tmem + C::TM_DPT + lane_off + c4 * 32, pv);
-        tmem_ld_wait(pv);
-        float p[32], ds[32];
+        tmem_ld32(tmem + C::TM_DP + lane_off + h * 32, dv);
+        tmem_ld_wait(dv);
+        float ds[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const int c = c4 * 32 + t;
-          float e = ex2(fmaf(__uint_as_float(sv[t]), sl2, -lse_s[c]));
-          if (diag && c < r) e = 0.f;
-          p[t] = e;
-          ds[t] = e * (__uint_as_float(pv[t]) - dvec_s[c]);
+          const int c = h * 32 + t;
+          float p = ex2(fmaf(__uint_as_float(sv[t]), sl2, -lse_s[c]));
+          if (diag && (q0 + c) < kv_idx) p = 0.f;
+          ds[t] = p * (__uint_as_float(dv[t]) - dvec_s[c]);
+          sv[t] = __float_as_uint(p);
         }
 #pragma unroll
+        for (int t = 0; t < 16; ++t)
+          pk[h * 16 + t] = pack_bf16x2(__uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]));
+#pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const int ch = c4 * 4 + q4;  // 16-byte chunk 0..15 along the 128 query columns
-          const uint32_t off = (ch >> 3) * 16384 + sw128_offset(r, ch & 7);
-          const int b = q4 * 8;
-          st_shared_v4(sPT + off, pack_bf16x2(p[b], p[b + 1]), pack_bf16x2(p[b + 2], p[b + 3]),
-                       pack_bf16x2(p[b + 4], p[b + 5]), pack_bf16x2(p[b + 6], p[b + 7]));
-          st_shared_v4(sDST + off, pack_bf16x2(ds[b], ds[b + 1]), pack_bf16x2(ds[b + 2], ds[b + 3]),
-                       pack_bf16x2(ds[b + 4], ds[b + 5]), pack_bf16x2(ds[b + 6], ds[b + 7]));
+          const int ch = h * 4 + q4;  // 16-byte chunk along the 64 query columns
+          st_shared_v4(sDS(b) + sw128_offset(r, ch), pack_bf16x2(ds[q4 * 8 + 0], ds[q4 * 8 + 1]),
+                       pack_bf16x2(ds[q4 * 8 + 2], ds[q4 * 8 + 3]), pack_bf16x2(ds[q4 * 8 + 4], ds[q4 * 8 + 5]),
+                       pack_bf16x2(ds[q4 * 8 + 6], ds[q4 * 8 + 7]));
+        }
+      }
+      tmem_st32(tS, pk);  // P^T (bf16) over the first 32 columns of this S buffer
+      tmem_st_wait();
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(bar_ds_full(b));
+    }
+    tc_fence_before();
+  } else if (warp < 8) {
+    // --------------------------------------------- dQ drain, dK/dV epilogue
+    const int wq = warp - 4;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const bool has_d = wq * 32 < D;  // TMEM lane = head-dim index of dQ^T
+    const int dcol = wq * 32 + lane;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      ok = mbar_wait(bar_dq_full, it & 1, abort_flag, kSiteBwdDrain);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      if (has_d) {
+        tmem_ld32(tmem + C::TM_DQ + lane_off, v0);
+        tmem_ld32(tmem + C::TM_DQ + lane_off + 32, v1);
+        tmem_ld_wait(v0);
+        tmem_ld_wait(v1);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dq_free);
+      if (has_d) {
+        float* dst = args.dq_acc + (size_t)(head_row0 + q_begin + it * C::BQ) * D + dcol;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) atomicAdd(dst + (size_t)c * D, __uint_as_float(v0[c]));
+#pragma unroll
+        for (int c = 0; c < 32; ++c) atomicAdd(dst + (size_t)(32 + c) * D, __uint_as_float(v1[c]));
+      }
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, kSiteBwdEpi));
+    if (ok) {
+      tc_fence_after();
+      // dV, dK rows (thread = key row) -> bf16 -> the now idle V and K tiles -> TMA store
+      const int row = wq * 32 + lane;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
+        const uint32_t sdst = which ? sK : sV;
+        const float mul = which ? args.scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tsrc + c * 32, v);
+          tmem_ld_wait(v);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int chunk = (c & 1) * 4 + q4;
+            const uint32_t* w = &v[q4 * 8];
+            st_shared_v4(sdst + (c >> 1) * C::KV_BLK + sw128_offset(row, chunk),
+                         pack_bf16x2(__uint_as_float(w[0]) * mul, __uint_as_float(w[1]) * mul),
+                         pack_bf16x2(__uint_as_float(w[2]) * mul, __uint_as_float(w[3]) * mul),
+                         pack_bf16x2(__uint_as_float(w[4]) * mul, __uint_as_float(w[5]) * mul),
+                         pack_bf16x2(__uint_as_float(w[6]) * mul, __uint_as_float(w[7]) * mul));
+          }
         }
       }
       fence_async_shared();
-      tc_fence_before();
-      mbar_arrive(bar_ds_full);
-      ok = mbar_wait(bar_dq_full, it & 1, abort_flag, kSiteBwdSoftDQ);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      // dQ_i partial (TMEM lane = query row r of tile i) -> fp32 atomics.
-      float* dst = args.dq_acc + ((size_t)(head_row0 + i * 128 + r)) * D;
+      named_barrier(1, 128);
+      if (wq == 0 && lane == 0) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + C::TM_DQ + lane_off + c * 32, v);
-        tmem_ld_wait(v);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int cc = (u + lane) & 7;  // rotate to spread the rows' addresses
-          atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + cc * 4),
-                    make_float4(__uint_as_float(v[cc * 4]), __uint_as_float(v[cc * 4 + 1]),
-                                __uint_as_float(v[cc * 4 + 2]), __uint_as_float(v[cc * 4 + 3])));
+        for (int kb = 0; kb < C::KB; ++kb) {
+          tma_store_2d(&tm_dv, sV + kb * C::KV_BLK, kb * 64, kv_row0);
+          tma_store_2d(&tm_dk, sK + kb * C::KV_BLK, kb * 64, kv_row0);
         }
-      }
-      tc_fence_before();
-      mbar_arrive(bar_tm_free);
-    }
-    if (ok) {
-      ok = mbar_wait(bar_done, 0, abort_flag, kSiteBwdEpi);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after();
-      const size_t row = (size_t)(kv_row0 + r) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + C::TM_DV + lane_off + c * 32, v);
-        tmem_ld_wait(v);
-        uint4* out = reinterpret_cast<uint4*>(args.dv + row + c * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const float* f = reinterpret_cast<const float*>(&v[q4 * 8]);
-          out[q4] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                               pack_bf16x2(f[6], f[7]));
-        }
-      }
-      const float sc = args.scale;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + C::TM_DK + lane_off + c * 32, v);
-        tmem_ld_wait(v);
-        uint4* out = reinterpret_cast<uint4*>(args.dk + row + c * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const float* f = reinterpret_cast<const float*>(&v[q4 * 8]);
-          out[q4] = make_uint4(pack_bf16x2(f[0] * sc, f[1] * sc), pack_bf16x2(f[2] * sc, f[3] * sc),
-                               pack_bf16x2(f[4] * sc, f[5] * sc), pack_bf16x2(f[6] * sc, f[7] * sc));
-        }
+        bulk_commit();
+        bulk_wait0();
       }
     }
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

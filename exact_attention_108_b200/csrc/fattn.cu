@@ -68,8 +68,9 @@ int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int ele
   return FATTN_OK;
 }
 
-int make_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int d) {
-  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, (uint64_t)d, 128, 64,
+// bf16 [rows, d] viewed in boxes of 64 columns x box_rows rows, 128-byte swizzle.
+int make_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int d, uint32_t box_rows = 128) {
+  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, (uint64_t)d, box_rows, 64,
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -111,12 +112,12 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <int D, bool CAUSAL>
 int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                const fattn::BwdArgs& a, int BH, cudaStream_t st) {
+                const CUtensorMap& mdk, const CUtensorMap& mdv, const fattn::BwdArgs& a, int BH, cudaStream_t st) {
   auto kern = fattn::fattn_bwd_dkdv_kernel<D, CAUSAL>;
   constexpr int smem = fattn::BwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
   dim3 grid((unsigned)((long long)BH * a.num_tiles));
-  kern<<<grid, 256, smem, st>>>(mq, mk, mv, mdo, a);
+  kern<<<grid, 320, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dkdv_kernel launch");
   return FATTN_OK;
@@ -153,23 +154,24 @@ template <int D>
 int launch_dkdv_d(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
                   int N, int causal, float scale, const WsParts& w, cudaStream_t st) {
   const long long rows = (long long)B * H * N;
-  CUtensorMap mq, mk, mv, mdo;
-  if (int rc = make_bf16_tile_map(&mq, q, rows, D)) return rc;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  if (int rc = make_bf16_tile_map(&mq, q, rows, D, fattn::BwdCfg<D>::BQ)) return rc;
+  if (int rc = make_bf16_tile_map(&mdo, dout, rows, D, fattn::BwdCfg<D>::BQ)) return rc;
   if (int rc = make_bf16_tile_map(&mk, k, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mv, v, rows, D)) return rc;
-  if (int rc = make_bf16_tile_map(&mdo, dout, rows, D)) return rc;
+  if (int rc = make_bf16_tile_map(&mdk, dk, rows, D)) return rc;
+  if (int rc = make_bf16_tile_map(&mdv, dv, rows, D)) return rc;
   fattn::BwdArgs a;
   a.lse2 = w.lse2;
   a.dvec = w.dvec;
   a.dq_acc = w.dq_acc;
-  a.dk = static_cast<__nv_bfloat16*>(dk);
-  a.dv = static_cast<__nv_bfloat16*>(dv);
   a.N = N;
   a.num_tiles = N / 128;
   a.scale = scale;
   a.scale_log2 = scale * kLog2e;
   const int BH = B * H;
-  return causal ? launch_dkdv<D, true>(mq, mk, mv, mdo, a, BH, st) : launch_dkdv<D, false>(mq, mk, mv, mdo, a, BH, st);
+  return causal ? launch_dkdv<D, true>(mq, mk, mv, mdo, mdk, mdv, a, BH, st)
+                : launch_dkdv<D, false>(mq, mk, mv, mdo, mdk, mdv, a, BH, st);
 }
 
 template <int D>
