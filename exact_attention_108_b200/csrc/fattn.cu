@@ -99,8 +99,8 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   auto kern = fattn::fattn_fwd_kernel<D, CAUSAL>;
   constexpr int smem = fattn::FwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
-  dim3 grid((unsigned)((long long)BH * a.num_q_tiles));
-  kern<<<grid, 256, smem, st>>>(mq, mk, mv, mo, a);
+  dim3 grid((unsigned)((long long)BH * ((a.num_q_tiles + 1) / 2)));
+  kern<<<grid, 384, smem, st>>>(mq, mk, mv, mo, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_fwd_kernel launch");
   return FATTN_OK;
