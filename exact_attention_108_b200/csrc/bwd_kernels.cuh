@@ -108,20 +108,21 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_STAT = OFF_DS + 2 * DS_BYTES;  // per stage: LSE2[64], D[64] fp32
   static constexpr int OFF_BAR = OFF_STAT + NS * 512;
-  // kv_full, q_full[NS], q_empty[NS], st_full[2], ds_full[2], pv_done[2], dq_full, dq_free, done, drain
-  static constexpr int NBAR = 1 + 2 * NS + 6 + 4;
+  // kv_full, q_full[NS], q_empty[NS], st_full[2], ds_full[2], dq_full[2], dq_free[2], done, drain
+  static constexpr int NBAR = 1 + 2 * NS + 8 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
-  // S^T buffers (P^T as bf16 overlays their first 32 columns), dP^T, dQ^T, dV, dK
-  static constexpr int TM_S0 = 0, TM_S1 = 64, TM_DP = 128, TM_DQ = 192, TM_DV = 256, TM_DK = 256 + D;
+  // Two 128-column regions R_b: S^T at +0 (P^T as bf16 overlays its first 32
+  // columns), dP^T at +64 (dQ^T of the same step replaces it once it has been
+  // read).  Then the dV and dK accumulators.
+  static constexpr int TM_R0 = 0, TM_R1 = 128, TM_DV = 256, TM_DK = 256 + D;
 };
 
 enum : int {
   kSiteBwdProducer = 0x201,
   kSiteBwdMmaKV = 0x202,
   kSiteBwdMmaQ = 0x203,
-  kSiteBwdMmaPV = 0x204,
   kSiteBwdMmaDS = 0x205,
   kSiteBwdMmaDQ = 0x206,
   kSiteBwdSoftS = 0x207,
@@ -158,9 +159,8 @@ __global__ void __launch_bounds__(320, 1)
   auto bar_q_empty = [&](int s) { return bar0 + 8u * (1 + C::NS + s); };
   auto bar_st_full = [&](int b) { return bar0 + 8u * (1 + 2 * C::NS + b); };
   auto bar_ds_full = [&](int b) { return bar0 + 8u * (3 + 2 * C::NS + b); };
-  auto bar_pv_done = [&](int b) { return bar0 + 8u * (5 + 2 * C::NS + b); };
-  const uint32_t bar_dq_full = bar0 + 8u * (7 + 2 * C::NS);
-  const uint32_t bar_dq_free = bar0 + 8u * (8 + 2 * C::NS);
+  auto bar_dq_full = [&](int b) { return bar0 + 8u * (5 + 2 * C::NS + b); };
+  auto bar_dq_free = [&](int b) { return bar0 + 8u * (7 + 2 * C::NS + b); };
   const uint32_t bar_done = bar0 + 8u * (9 + 2 * C::NS);
   const uint32_t bar_drain = bar0 + 8u * (10 + 2 * C::NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -188,10 +188,9 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_st_full(b), 1);
       mbar_init(bar_ds_full(b), 128);
-      mbar_init(bar_pv_done(b), 1);
+      mbar_init(bar_dq_full(b), 1);
+      mbar_init(bar_dq_free(b), 128);
     }
-    mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 128);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -250,55 +249,60 @@ __global__ void __launch_bounds__(320, 1)
       // A repeats the first (LBO = 0) and its output lanes are ignored.
       constexpr uint32_t kt_lbo = (D == 128) ? C::KV_BLK : 0;
       bool ok = mbar_wait(bar_kv_full, 0, abort_flag, kSiteBwdMmaKV);
-      auto issue_s_dp = [&](int it) -> bool {
-        const int s = it % C::NS, b = it & 1;
+      auto region = [&](int b) { return tmem + (b ? C::TM_R1 : C::TM_R0); };
+      auto issue_s_dp = [&](int it) -> bool {  // S^T, dP^T of step `it` into region it % 2
+        const int s = it % C::NS;
         if (!mbar_wait(bar_q_full(s), (it / C::NS) & 1, abort_flag, kSiteBwdMmaQ)) return false;
-        // P^T of iteration it-2 lives in this S buffer: its dV product must be done
-        if (it >= 2 && !mbar_wait(bar_pv_done(b), ((it >> 1) & 1) ^ 1, abort_flag, kSiteBwdMmaPV)) return false;
         tc_fence_after();
-        const uint32_t tS = tmem + (b ? C::TM_S1 : C::TM_S0);
+        const uint32_t R = region(it & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * C::KV_BLK + (kk & 3) * 32;
           const uint32_t kb = (kk >> 2) * C::Q_BLK + (kk & 3) * 32;
-          mma_ss(tS, sdesc_sw128(sK + ka, 16), sdesc_sw128(sQ(s) + kb, 16), id_s, kk > 0);
+          mma_ss(R, sdesc_sw128(sK + ka, 16), sdesc_sw128(sQ(s) + kb, 16), id_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * C::KV_BLK + (kk & 3) * 32;
           const uint32_t kb = (kk >> 2) * C::Q_BLK + (kk & 3) * 32;
-          mma_ss(tmem + C::TM_DP, sdesc_sw128(sV + ka, 16), sdesc_sw128(sDO(s) + kb, 16), id_s, kk > 0);
+          mma_ss(R + 64, sdesc_sw128(sV + ka, 16), sdesc_sw128(sDO(s) + kb, 16), id_s, kk > 0);
         }
-        mma_commit(bar_st_full(b));
+        mma_commit(bar_st_full(it & 1));
         return true;
       };
+      // Tensor-core order: S,dP(0) S,dP(1) | dV,dK,dQ(0) S,dP(2) | dV,dK,dQ(1) S,dP(3) | ...
+      // so that the softmax-gradient group works on step i+1 while the tensor
+      // cores run the five products of steps i and i+2.
       if (ok) ok = issue_s_dp(0);
+      if (ok && n_it > 1) ok = issue_s_dp(1);
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it % C::NS, b = it & 1;
         if (!(ok = mbar_wait(bar_ds_full(b), (it >> 1) & 1, abort_flag, kSiteBwdMmaDS))) break;
         tc_fence_after();
-        if (it + 1 < n_it && !(ok = issue_s_dp(it + 1))) break;
-        const uint32_t tP = tmem + (b ? C::TM_S1 : C::TM_S0);
+        const uint32_t R = region(b);
         // dV += P^T dO  (A = P^T from TMEM: 4 x 16 query columns, 8 TMEM columns each)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts(tmem + C::TM_DV, tP + kk * 8, sdesc_sw128(sDO(s) + kk * 2048, C::Q_BLK), id_kv,
+          mma_ts(tmem + C::TM_DV, R + kk * 8, sdesc_sw128(sDO(s) + kk * 2048, C::Q_BLK), id_kv,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_pv_done(b));
         // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           mma_ss(tmem + C::TM_DK, sdesc_sw128(sDS(b) + kk * 32, 16), sdesc_sw128(sQ(s) + kk * 2048, C::Q_BLK),
                  id_kv, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_q_empty(s));
-        // dQ^T = K^T dS^T once the previous dQ^T has been drained
-        if (!(ok = mbar_wait(bar_dq_free, (it & 1) ^ 1, abort_flag, kSiteBwdMmaDQ))) break;
-        tc_fence_after();
+        // dQ^T = K^T dS^T into the dP^T half of this region (already read)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + C::TM_DQ, sdesc_sw128(sK + kk * 2048, kt_lbo), sdesc_sw128(sDS(b) + kk * 2048, 16), id_q,
+          mma_ss(R + 64, sdesc_sw128(sK + kk * 2048, kt_lbo), sdesc_sw128(sDS(b) + kk * 2048, 16), id_q,
                  kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq_full);
+        mma_commit(bar_dq_full(b));
+        if (it + 2 < n_it) {
+          // region b is free once dQ^T(it) has been drained (which also implies that
+          // dV(it), the reader of P^T, has completed)
+          if (!(ok = mbar_wait(bar_dq_free(b), (it >> 1) & 1, abort_flag, kSiteBwdMmaDQ))) break;
+          if (!(ok = issue_s_dp(it + 2))) break;
+        }
       }
       if (ok) mma_commit(bar_done);
       mma_commit(bar_drain);
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(320, 1)
       ok = ok && mbar_wait(bar_q_full(s), (it / C::NS) & 1, abort_flag, kSiteBwdSoftQ);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const uint32_t tS = tmem + (b ? C::TM_S1 : C::TM_S0) + lane_off;
+      const uint32_t tS = tmem + (b ? C::TM_R1 : C::TM_R0) + lane_off;
       const float* lse_s = stat(s);
       const float* dvec_s = stat(s) + 64;
       const int q0 = q_begin + it * C::BQ;  // first query row (in the head) of this sub-tile
@@ -328,7 +332,7 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + h * 32, sv);
         tmem_ld_wait(sv);
-        tmem_ld32(tmem + C::TM_DP + lane_off + h * 32, dv);
+        tmem_ld32(tS + 64 + h * 32, dv);
         tmem_ld_wait(dv);
         float ds[32];
 #pragma unroll
@@ -365,18 +369,20 @@ __global__ void __launch_bounds__(320, 1)
     const int dcol = wq * 32 + lane;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      ok = mbar_wait(bar_dq_full, it & 1, abort_flag, kSiteBwdDrain);
+      const int b = it & 1;
+      ok = mbar_wait(bar_dq_full(b), (it >> 1) & 1, abort_flag, kSiteBwdDrain);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
+      const uint32_t tDQ = tmem + (b ? C::TM_R1 : C::TM_R0) + 64 + lane_off;
       uint32_t v0[32], v1[32];
       if (has_d) {
-        tmem_ld32(tmem + C::TM_DQ + lane_off, v0);
-        tmem_ld32(tmem + C::TM_DQ + lane_off + 32, v1);
+        tmem_ld32(tDQ, v0);
+        tmem_ld32(tDQ + 32, v1);
         tmem_ld_wait(v0);
         tmem_ld_wait(v1);
       }
       tc_fence_before();
-      mbar_arrive(bar_dq_free);
+      mbar_arrive(bar_dq_free(b));
       if (has_d) {
         float* dst = args.dq_acc + (size_t)(head_row0 + q_begin + it * C::BQ) * D + dcol;
 #pragma unroll
