@@ -15,6 +15,19 @@
 #include "bwd_kernels.cuh"
 #include "fwd_kernel.cuh"
 
+namespace fattn {
+__global__ void fattn_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  for (long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x); i < n;
+       i += 2ll * gridDim.x * blockDim.x) {
+    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
+    float y0, y1;
+    sm100::f2_unpack(sm100::exp2_poly_x2(sm100::f2_pack(x0, x1)), y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+  }
+}
+}  // namespace fattn
+
 namespace {
 
 thread_local std::string t_last_cuda_error;
@@ -259,6 +272,19 @@ int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, 
                              : launch_fwd<64, false>(mq, mk, mv, mo, a, BH, st);
   return causal ? launch_fwd<128, true>(mq, mk, mv, mo, a, BH, st)
                 : launch_fwd<128, false>(mq, mk, mv, mo, a, BH, st);
+}
+
+int fattn_exp2_poly(const float* x, float* y, long long n, fattn_stream_t stream) {
+  if (n < 0 || ((!x || !y) && n > 0)) return FATTN_ERR_INVALID_ARG;
+  if (n == 0) return FATTN_OK;
+  if (!aligned16(x) || !aligned16(y)) return FATTN_ERR_ALIGNMENT;
+  long long blocks = (n / 2 + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks < 1) blocks = 1;
+  fattn::fattn_exp2_poly_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_exp2_poly_kernel launch");
+  return FATTN_OK;
 }
 
 size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {

@@ -59,6 +59,10 @@ struct FwdCfg {
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: weights stay below 256
+// Exponentials evaluated on the FMA pipe (exp2_poly_x2) per 8 pairs of columns;
+// the rest use MUFU ex2.  On B200 at this tile shape the extra FMA-pipe
+// instructions cost about what they save on MUFU, so the share is 0.
+constexpr int kPolyPairsPer8 = 0;
 
 enum : int {  // wait sites recorded in the device status word on a timeout
   kSiteFwdProducer = 0x101,
@@ -266,18 +270,32 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 128; ++c)
           if (c > r) v[c >> 5][c & 31] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
       }
-      // row max of the raw scores, turned into the max of scale * score (log2 units)
+      // row max of the raw scores, turned into the max of scale * score (log2 units);
+      // four independent three-input chains keep the dependencies short
       float mx;
-      if (sl2 >= 0.f) {
-        mx = -INFINITY;
+      {
+        float pm[4];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(v[c >> 5][c & 31]));
-      } else {
-        mx = INFINITY;
+        for (int u = 0; u < 4; ++u) pm[u] = __uint_as_float(v[u][0]);
+        if (sl2 >= 0.f) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fminf(mx, __uint_as_float(v[c >> 5][c & 31]));
+          for (int c = 0; c < 128; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                            __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+          mx = fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                            __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+          mx = fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
+        }
+        mx *= sl2;
       }
-      mx *= sl2;
       // lazily move the reference max; rescale O and l only when it moves
       const bool grow = mx > m_ref + kRescaleThreshold;
       if (__any_sync(0xffffffffu, grow)) {
@@ -297,22 +315,37 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      const float neg_m = -m_ref;
       const bool diag = CAUSAL && j == q_tile;  // keys c > r of this tile are masked
-      float sum = 0.f;
-      uint32_t pk[2][32];  // P row as packed bf16 pairs
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
+      uint32_t pk[2][32];                          // P row as packed bf16 pairs
 #pragma unroll
       for (int c = 0; c < 128; c += 2) {
-        float p0 = ex2(fmaf(__uint_as_float(v[c >> 5][c & 31]), sl2, neg_m));
-        float p1 = ex2(fmaf(__uint_as_float(v[(c + 1) >> 5][(c + 1) & 31]), sl2, neg_m));
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
+                                           __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
+                                   sl2x2, negm2);
+        float p0, p1;
+        if (((c >> 1) & 7) < kPolyPairsPer8) {
+          f2_unpack(exp2_poly_x2(x2), p0, p1);  // on the FMA pipe
+        } else {
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          p0 = ex2(x0);
+          p1 = ex2(x1);
+        }
         if (diag) {
           p0 = (c > r) ? 0.f : p0;
           p1 = (c + 1 > r) ? 0.f : p1;
         }
-        sum += p0 + p1;
+        acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
         pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
       }
-      l += sum;
+      {
+        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float s0, s1;
+        f2_unpack(a2, s0, s1);
+        l += s0 + s1;
+      }
       // P (bf16 pairs) over the first 64 columns of S_k
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);

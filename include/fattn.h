@@ -114,6 +114,17 @@ int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout
 int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale,
                  void* workspace, size_t workspace_bytes, fattn_stream_t stream);
 
+/*
+ * Diagnostics: y[i] = 2^x[i] evaluated with the FMA-pipe approximation the
+ * softmax loops can use for part of their exponentials to offload the MUFU
+ * unit (range reduction to n + f, f in [-1/2, 1/2], degree-3 minimax
+ * polynomial for 2^f; relative error <= 1.1e-4 for x >= -64, inputs below -64
+ * are treated as -64).
+ * x, y: device fp32 arrays of n elements, 16-byte aligned, n >= 0.
+ * Exposed so that the approximation's error bound can be tested on the GPU.
+ */
+int fattn_exp2_poly(const float* x, float* y, long long n, fattn_stream_t stream);
+
 /* Static, human-readable text for a status code. */
 const char* fattn_status_string(int status);
 
