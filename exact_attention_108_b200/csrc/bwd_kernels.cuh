@@ -14,7 +14,7 @@
 //                              P^T  = exp2(S^T scale log2e - LSE2_i)   (masked)
 //                              dS^T = P^T o (dP^T - D_i)
 //                              dV_j += P^T dO_i   (P^T read from TMEM)
-//                              dK_j += dS^T Q_i   (TMEM accumulators)
+//                              dK_j += dS^T Q_i   (dS^T read from TMEM)
 //                              dQ_i^T = K_j^T dS^T_i -> fp32 atomics into the
 //                                                       accumulator
 //                            (atomic global updates, page 3 "5.3 专用指令利用").
@@ -113,9 +113,9 @@ struct BwdCfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
-  // Two 128-column regions R_b: S^T at +0 (P^T as bf16 overlays its first 32
-  // columns), dP^T at +64 (dQ^T of the same step replaces it once it has been
-  // read).  Then the dV and dK accumulators.
+  // Two 128-column regions R_b: S^T at +0 (once read, P^T and dS^T as bf16
+  // pairs overlay its columns 0..31 and 32..63), dP^T at +64 (dQ^T of the same
+  // step replaces it once it has been read).  Then the dV and dK accumulators.
   static constexpr int TM_R0 = 0, TM_R1 = 128, TM_DV = 256, TM_DK = 256 + D;
 };
 
@@ -285,11 +285,11 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           mma_ts(tmem + C::TM_DV, R + kk * 8, sdesc_sw128(sDO(s) + kk * 2048, C::Q_BLK), id_kv,
                  (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q
+        // dK += dS^T Q  (A = dS^T from TMEM, columns 32..63 of the region)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ss(tmem + C::TM_DK, sdesc_sw128(sDS(b) + kk * 32, 16), sdesc_sw128(sQ(s) + kk * 2048, C::Q_BLK),
-                 id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::TM_DK, R + 32 + kk * 8, sdesc_sw128(sQ(s) + kk * 2048, C::Q_BLK), id_kv,
+                 (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_q_empty(s));
         // dQ^T = K^T dS^T into the dP^T half of this region (already read)
 #pragma unroll
@@ -326,7 +326,8 @@ __global__ void __launch_bounds__(320, 1)
       const float* dvec_s = stat(s) + 64;
       const int q0 = q_begin + it * C::BQ;  // first query row (in the head) of this sub-tile
       const bool diag = CAUSAL && (q0 < kv_tile * 128 + 128);
-      uint32_t pk[32];  // P^T row, packed bf16 pairs
+      uint32_t pk[32];   // P^T row, packed bf16 pairs
+      uint32_t dsk[32];  // dS^T row, packed bf16 pairs
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t sv[32], dv[32];
@@ -344,17 +345,19 @@ __global__ void __launch_bounds__(320, 1)
           sv[t] = __float_as_uint(p);
         }
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
+        for (int t = 0; t < 16; ++t) {
           pk[h * 16 + t] = pack_bf16x2(__uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]));
+          dsk[h * 16 + t] = pack_bf16x2(ds[2 * t], ds[2 * t + 1]);
+        }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int ch = h * 4 + q4;  // 16-byte chunk along the 64 query columns
-          st_shared_v4(sDS(b) + sw128_offset(r, ch), pack_bf16x2(ds[q4 * 8 + 0], ds[q4 * 8 + 1]),
-                       pack_bf16x2(ds[q4 * 8 + 2], ds[q4 * 8 + 3]), pack_bf16x2(ds[q4 * 8 + 4], ds[q4 * 8 + 5]),
-                       pack_bf16x2(ds[q4 * 8 + 6], ds[q4 * 8 + 7]));
+          const uint32_t* w = &dsk[h * 16 + q4 * 4];
+          st_shared_v4(sDS(b) + sw128_offset(r, ch), w[0], w[1], w[2], w[3]);
         }
       }
-      tmem_st32(tS, pk);  // P^T (bf16) over the first 32 columns of this S buffer
+      tmem_st32(tS, pk);        // P^T (bf16) over columns 0..31 of this region
+      tmem_st32(tS + 32, dsk);  // dS^T (bf16) over columns 32..63 (S^T already read)
       tmem_st_wait();
       fence_async_shared();
       tc_fence_before();
