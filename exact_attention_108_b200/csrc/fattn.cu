@@ -130,7 +130,7 @@ int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   constexpr int smem = fattn::BwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
   dim3 grid((unsigned)((long long)BH * a.num_tiles));
-  kern<<<grid, 320, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, a);
+  kern<<<grid, 384, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dkdv_kernel launch");
   return FATTN_OK;
@@ -168,8 +168,8 @@ int launch_dkdv_d(const void* q, const void* k, const void* v, const void* dout,
                   int N, int causal, float scale, const WsParts& w, cudaStream_t st) {
   const long long rows = (long long)B * H * N;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if (int rc = make_bf16_tile_map(&mq, q, rows, D, fattn::BwdCfg<D>::BQ)) return rc;
-  if (int rc = make_bf16_tile_map(&mdo, dout, rows, D, fattn::BwdCfg<D>::BQ)) return rc;
+  if (int rc = make_bf16_tile_map(&mq, q, rows, D)) return rc;
+  if (int rc = make_bf16_tile_map(&mdo, dout, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mk, k, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mv, v, rows, D)) return rc;
   if (int rc = make_bf16_tile_map(&mdk, dk, rows, D)) return rc;
