@@ -339,9 +339,14 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) tmem_ld_wait(v[c4]);
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float e = ex2(fmaf(__uint_as_float(v[c >> 5][c & 31]), sl2, -lse_s[c]));
-          p[c] = (diag && c < r) ? 0.f : e;
+        for (int c = 0; c < 128; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c);  // one broadcast load per 4 columns
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float e = ex2(fmaf(__uint_as_float(v[(c + u) >> 5][(c + u) & 31]), sl2, -lv[u]));
+            p[c + u] = (diag && c + u < r) ? 0.f : e;
+          }
         }
       }
       {
@@ -365,10 +370,13 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld_wait(dv);
         uint32_t dsk[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
+        for (int t = 0; t < 16; t += 2) {
           const int c = c4 * 32 + 2 * t;
-          dsk[t] = pack_bf16x2(p[c] * (__uint_as_float(dv[2 * t]) - dvec_s[c]),
-                               p[c + 1] * (__uint_as_float(dv[2 * t + 1]) - dvec_s[c + 1]));
+          const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c);  // one broadcast load per 4 columns
+          dsk[t] = pack_bf16x2(p[c] * (__uint_as_float(dv[2 * t]) - d4.x),
+                               p[c + 1] * (__uint_as_float(dv[2 * t + 1]) - d4.y));
+          dsk[t + 1] = pack_bf16x2(p[c + 2] * (__uint_as_float(dv[2 * t + 2]) - d4.z),
+                                   p[c + 3] * (__uint_as_float(dv[2 * t + 3]) - d4.w));
         }
         tmem_st16(tA + 64 + c4 * 16, dsk);
 #pragma unroll
