@@ -21,11 +21,13 @@ FATTN_ERR_UNSUPPORTED = 2
 FATTN_ERR_ALIGNMENT = 3
 FATTN_ERR_CUDA = 4
 FATTN_ERR_DEVICE_TIMEOUT = 5
+FATTN_ERR_SCRATCH_TOO_SMALL = 6
+NOALLOC_SCRATCH_BYTES = 32 << 20  # FATTN_NOALLOC_SCRATCH_BYTES
 
 # Every symbol include/fattn.h declares (checked by the CPU test suite).
 EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_bwd_preprocess",
             "fattn_bwd_dkdv", "fattn_bwd_dq", "fattn_status_string", "fattn_last_cuda_error",
-            "fattn_device_status", "fattn_version", "fattn_exp2_poly")
+            "fattn_device_status", "fattn_version", "fattn_exp2_poly", "fattn_bwd_noalloc")
 
 _lib = None
 
@@ -52,6 +54,8 @@ def load():
     L.fattn_fwd.restype = i
     L.fattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     L.fattn_bwd.restype = i
+    L.fattn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    L.fattn_bwd_noalloc.restype = i
     L.fattn_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
     L.fattn_bwd_preprocess.restype = i
     L.fattn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
@@ -201,3 +205,32 @@ def exp2_poly(x, out=None, stream=None):
     if rc != FATTN_OK:
         raise FattnError(rc, "fattn_exp2_poly")
     return out
+
+
+def bwd_noalloc(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
+                dq=None, dk=None, dv=None, stream=None):
+    """The backward without any workspace: for callers that cannot allocate device
+    memory or hand the library a buffer (see fattn_bwd_noalloc in include/fattn.h).
+
+    Results are those of bwd(); the scratch comes from a fixed 32 MiB array the
+    library keeps on each device, so larger shapes raise FattnError and calls that
+    overlap on the GPU must not share a device.  (dq, dk, dv are created here when
+    not given, as in bwd(); pass them to keep this wrapper allocation-free too.)
+    """
+    B, H, N, d = _shape4(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n)
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{n} has shape {tuple(t.shape)}, expected {(B, H, N, d)}")
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = load().fattn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                  lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                  B, H, N, d, 1 if causal else 0, float(scale), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_bwd_noalloc")
+    return dq, dk, dv

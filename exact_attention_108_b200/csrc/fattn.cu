@@ -227,6 +227,8 @@ const char* fattn_status_string(int status) {
     case FATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case FATTN_ERR_CUDA: return "CUDA error (see fattn_last_cuda_error)";
     case FATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";
+    case FATTN_ERR_SCRATCH_TOO_SMALL:
+      return "shape needs more scratch than fattn_bwd_noalloc has (FATTN_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }
@@ -344,6 +346,49 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o, const 
   if (int rc = fattn_bwd_dkdv(q, k, v, dout, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes, stream))
     return rc;
   return fattn_bwd_dq(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// fattn_bwd_noalloc: the backward's scratch lives in this fixed device array
+// instead of a caller-provided workspace.  In host code the array's name only
+// stands for the symbol; its device address comes from cudaGetSymbolAddress,
+// looked up once per device (with that device current) and cached.
+static __device__ __align__(256) unsigned char g_fattn_noalloc_scratch[FATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch_ptr[256] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 256) {
+    t_last_cuda_error = "device ordinal out of range for the no-allocation scratch table";
+    return FATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fattn_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    g_noalloc_scratch_ptr[dev] = p;
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return FATTN_OK;
+}
+}  // namespace
+
+int fattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                      void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
+                      fattn_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_common(B, H, N, d, scale, causal)) return rc;
+  if (fattn_bwd_workspace_size(B, H, N, d) > (size_t)FATTN_NOALLOC_SCRATCH_BYTES) return FATTN_ERR_SCRATCH_TOO_SMALL;
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  return fattn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, scratch,
+                   (size_t)FATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

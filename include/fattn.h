@@ -60,7 +60,8 @@ typedef enum {
   FATTN_ERR_UNSUPPORTED = 2,    /* d not in {64,128}, N % 128 != 0, size overflow */
   FATTN_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
   FATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed; see fattn_last_cuda_error() */
-  FATTN_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out */
+  FATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out */
+  FATTN_ERR_SCRATCH_TOO_SMALL = 6 /* fattn_bwd_noalloc: the shape needs more than its fixed scratch */
 } fattn_status;
 
 /*
@@ -92,6 +93,37 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o,
               const void* dout, const float* lse, void* dq, void* dk, void* dv,
               int B, int H, int N, int d, int causal, float scale,
               void* workspace, size_t workspace_bytes, fattn_stream_t stream);
+
+/*
+ * Backward that allocates nothing and takes no workspace argument.
+ *
+ * The pages the library follows have no counterpart of this call.  It is for
+ * callers that cannot allocate device memory or hand over a buffer of their
+ * own: for example a plugin running inside a host application that owns all
+ * device memory and gives the plugin no allocator, or a serving loop that
+ * reserves its memory once at start-up and forbids allocations (and the
+ * device-wide synchronisation an allocation can cause) on its request path.
+ *
+ * Arguments, layout, results and errors are those of fattn_bwd without the
+ * workspace.  The scratch space fattn_bwd takes from its workspace comes
+ * instead from one fixed array of FATTN_NOALLOC_SCRATCH_BYTES bytes (32 MiB)
+ * that the library keeps in device memory; every GPU that loads the library
+ * holds that array until the process exits.  Shapes whose workspace
+ * (fattn_bwd_workspace_size) is larger are rejected with
+ * FATTN_ERR_SCRATCH_TOO_SMALL before anything is enqueued: at d = 128 that is
+ * B*H*N > 64512, at d = 64 B*H*N > 126976.
+ *
+ * The first call on a device looks up the array's device address and caches
+ * it; make that first call before any stream capture on that device.  All calls
+ * on one device share the array, and each call re-initialises what must start
+ * at zero, so calls whose executions overlap on the GPU (on different streams,
+ * or from several host threads) race on it and must be serialised by the caller.
+ */
+#define FATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+int fattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      int B, int H, int N, int d, int causal, float scale,
+                      fattn_stream_t stream);
 
 /*
  * The three stages fattn_bwd runs, exposed so that callers can schedule or time
