@@ -5,8 +5,8 @@
 One step = one pass of the whole hot path over one batch: fattn_fwd (O, LSE)
 followed by the three backward stages (preprocess, dK/dV with dQ atomics, dQ
 convert).  The default workload is the d=128 causal training shape
-B=4, H=32, N=4096.  Every input tensor (256 MiB each) is larger than the 126 MB
-L2, so no flush is needed between steps.
+B=4, H=32, N=4096.  Each step reads Q, K, V, dO and O (640 MiB at the default
+shape), far more than the 126 MB L2, so no flush is needed between steps.
 
 Multi-GPU (torchrun): each rank runs the same step on its own batch drawn with
 seed + rank (independent problems, no collective on the data path: weak
@@ -354,8 +354,8 @@ def run_fattn(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "dist": w.dist, "global_batch": w.B * world,
-                   "l2": "inputs larger than L2 (each of Q,K,V,dO,O is "
-                         f"{w.B * w.H * w.N * w.d * 2 / 2**20:.0f} MiB > 126 MB); no flush"},
+                   "l2": "inputs larger than L2: each step reads Q, K, V, dO and O, "
+                         f"{5 * w.B * w.H * w.N * w.d * 2 / 2**20:.0f} MiB in all (> 126 MB L2); no flush"},
         "fwd_tflops": round(fwd_tflops, 1), "bwd_tflops": round(bwd_tflops, 1),
         "fwd_frac_of_peak": round(fwd_tflops / peak, 4), "bwd_frac_of_peak": round(bwd_tflops / peak, 4),
         "stage_ms": {"fwd": round(fwd_ms, 4), "bwd_preprocess": round(pre_ms, 4),
