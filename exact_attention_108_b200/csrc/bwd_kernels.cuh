@@ -15,8 +15,9 @@
 //                              dS^T = P^T o (dP^T - D_i)
 //                              dV_j += P^T dO_i   (P^T read from TMEM)
 //                              dK_j += dS^T Q_i   (dS^T read from TMEM)
-//                              dQ_i^T = K_j^T dS^T_i -> fp32 atomics into the
-//                                                       accumulator
+//                              dQ_i^T = K_j^T dS^T_i -> staged in shared memory,
+//                                  added into the fp32 accumulator by one TMA
+//                                  bulk reduce per query tile
 //                            (atomic global updates, page 3 "5.3 专用指令利用").
 //  3. fattn_bwd_dq_kernel    dQ = bf16(scale * accumulator).
 #pragma once
@@ -104,8 +105,9 @@ struct BwdCfg {
   static constexpr int STAGE = 2 * TILE + 1024;  // Q tile, dO tile, LSE2[128], D[128]
   static constexpr int OFF_DS = OFF_STAGE + NS * STAGE;
   static constexpr int OFF_BAR = OFF_DS + DS_BYTES;
-  // kv_full, q_full[NS], q_empty[NS], s_full, dp_full, p_full, ds_full, dq_full, dq_free, done, drain
-  static constexpr int NBAR = 1 + 2 * NS + 8;
+  // kv_full, q_full[NS], q_empty[NS], s_full, dp_full, p_full, ds_full, dq_full, dq_free, done, drain,
+  // staged (dQ partial written to shared memory)
+  static constexpr int NBAR = 1 + 2 * NS + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;  // the dynamic shared window starts 1024-byte aligned
   static constexpr int TMEM_COLS = 512;
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t bar_s_full = bar0 + 8u * (1 + 2 * C::NS);
   const uint32_t bar_dp_full = bar_s_full + 8, bar_p_full = bar_s_full + 16, bar_ds_full = bar_s_full + 24;
   const uint32_t bar_dq_full = bar_s_full + 32, bar_dq_free = bar_s_full + 40, bar_done = bar_s_full + 48;
-  const uint32_t bar_drain = bar_s_full + 56;
+  const uint32_t bar_drain = bar_s_full + 56, bar_staged = bar_s_full + 64;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar_dq_free, 128);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_staged, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + C::TM_DK, tA + 64 + kk * 8, sdesc_sw128(sQ(s) + kk * 2048, C::BLK), id_kv,
                    (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar_q_empty(s));
+          // (the Q/dO stage is released by the dQ drain, which reuses it as staging)
           // dQ^T = K^T dS^T into region B (dP^T already read)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -413,12 +416,31 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_fence_before();
       mbar_arrive(bar_dq_free);
+      // dQ^T_i -> shared memory as row-major fp32 [128 queries][D] in this step's Q/dO
+      // stage (free: its last readers, dV_i and dK_i, completed before dQ^T_i) ->
+      // one TMA bulk reduce-add into the accumulator rows, which are contiguous.
+      const int s = it % C::NS;
       if (has_d) {
-        float* dst = args.dq_acc + (size_t)(head_row0 + (i_begin + it) * 128) * D + dcol;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) atomicAdd(dst + (size_t)c * D, __uint_as_float(v[c >> 5][c & 31]));
+        for (int c = 0; c < 128; ++c)
+          st_shared_f32(sQ(s) + (uint32_t)(c * D + dcol) * 4u, __uint_as_float(v[c >> 5][c & 31]));
       }
+      fence_async_shared();
+      mbar_arrive(bar_staged);
+      if (wq == 0 && lane == 0) {
+        ok = mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain);
+        if (ok) {
+          float* dst = args.dq_acc + (size_t)(head_row0 + (i_begin + it) * 128) * D;
+          bulk_reduce_add_f32(dst, sQ(s), 128 * D * 4);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        mbar_arrive(bar_q_empty(s));  // the producer may refill the stage
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
     }
+    if (wq == 0 && lane == 0) bulk_wait0();  // the last reduce has landed in global memory
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, kSiteBwdEpi));
     if (ok) {
       tc_fence_after();
