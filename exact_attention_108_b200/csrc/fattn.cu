@@ -95,7 +95,7 @@ int check_shape(int B, int H, int N, int d) {
   if (N % 128 != 0) return FATTN_ERR_UNSUPPORTED;
   const long long rows = (long long)B * H * N;
   if (rows >= (1ll << 31)) return FATTN_ERR_UNSUPPORTED;
-  if (rows / 128 > 0x7fffffffll) return FATTN_ERR_UNSUPPORTED;  // one CTA per 128-row tile
+  if (rows / 128 > 0x7fffffffll) return FATTN_ERR_UNSUPPORTED;  // 128-row tiles are counted in int
   return FATTN_OK;
 }
 
@@ -106,16 +106,134 @@ int set_smem(K kernel, int bytes) {
   return FATTN_OK;
 }
 
+constexpr int kMaxDevices = 256;
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (*dev < 0 || *dev >= kMaxDevices) {
+    t_last_cuda_error = "device ordinal out of range";
+    return FATTN_ERR_CUDA;
+  }
+  return FATTN_OK;
+}
+
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count(int* out) {
+  static std::mutex mu;
+  static int counts[kMaxDevices] = {};
+  int dev = 0;
+  if (int rc = current_device(&dev)) return rc;
+  cudaError_t e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!counts[dev]) {
+    e = cudaDeviceGetAttribute(&counts[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  *out = counts[dev];
+  return FATTN_OK;
+}
+
+// Causal forward: the heads' scheduling groups.  The units of a group run
+// longest first, so a group must hold enough work that its longest unit (N/128
+// key tiles) is no more than about 2/3 of what each SM gets from the group; its
+// keys and values (4*N*d bytes per head) should stay well inside L2.  The heads
+// are then split into groups whose sizes differ by at most one (a small last
+// group would leave its long units running alone at the end).
+void causal_groups(int BH, int N, int d, int sms, int* big, int* num_big) {
+  const long long nt = N / 128, np = (nt + 1) / 2;
+  long long work = 0;  // key tiles summed over the pairs of one head
+  for (long long p = 0; p < np; ++p) work += (2 * p + 2 < nt ? 2 * p + 2 : nt);
+  long long g = (3ll * sms * nt + 2 * work - 1) / (2 * work);
+  const long long cap = (48ll << 20) / (4ll * N * d);
+  if (g > cap) g = cap;
+  if (g > BH) g = BH;
+  if (g < 1) g = 1;
+  const int ng = (int)(BH / g), q = BH / ng, r = BH % ng;
+  *big = r ? q + 1 : q;
+  *num_big = r ? r : ng;
+}
+
+// Counters for the causal forward's dynamic unit claiming, kSchedSlots pairs per
+// device.  A slot goes to a launch only once the event recorded after the slot's
+// previous launch has completed -- that launch's last CTA has returned the
+// counters to 0 -- so no two kernels in flight share one.  A launch being
+// captured into a CUDA graph, or one that finds every slot busy, schedules its
+// units statically instead.
+constexpr int kSchedSlots = 16;
+static __device__ unsigned int g_fwd_sched[kSchedSlots][2];
+
+struct SchedPool {
+  std::mutex mu;
+  bool ready = false;
+  unsigned int* base = nullptr;
+  cudaEvent_t ev[kSchedSlots] = {};
+  int next = 0;
+};
+SchedPool g_sched_pool[kMaxDevices];
+
+// Picks a free slot (pool locked by the caller); -1 if none is usable.
+int sched_slot(SchedPool& pool, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  if (cs != cudaStreamCaptureStatusNone) return -1;
+  if (!pool.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fwd_sched) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return -1;
+    }
+    for (int i = 0; i < kSchedSlots; ++i)
+      if (cudaEventCreateWithFlags(&pool.ev[i], cudaEventDisableTiming) != cudaSuccess) {
+        (void)cudaGetLastError();
+        for (int j = 0; j < i; ++j) cudaEventDestroy(pool.ev[j]);
+        return -1;
+      }
+    pool.base = static_cast<unsigned int*>(p);
+    pool.ready = true;
+  }
+  for (int i = 0; i < kSchedSlots; ++i) {
+    const int s = (pool.next + i) % kSchedSlots;
+    if (cudaEventQuery(pool.ev[s]) == cudaSuccess) {
+      pool.next = (s + 1) % kSchedSlots;
+      return s;
+    }
+  }
+  return -1;
+}
+
 template <int D, bool CAUSAL>
-int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
-               const fattn::FwdArgs& a, int BH, cudaStream_t st) {
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fattn::FwdArgs& a,
+               cudaStream_t st) {
   auto kern = fattn::fattn_fwd_kernel<D, CAUSAL>;
   constexpr int smem = fattn::FwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
-  dim3 grid((unsigned)((long long)BH * ((a.num_q_tiles + 1) / 2)));
-  kern<<<grid, 384, smem, st>>>(mq, mk, mv, mo, a);
+  int sms = 0, dev = 0;
+  if (int rc = sm_count(&sms)) return rc;
+  if (int rc = current_device(&dev)) return rc;
+  const int ctas = a.num_units < sms ? a.num_units : sms;  // persistent: at most one CTA per SM
+  fattn::FwdArgs args = a;
+  args.sched = nullptr;
+  if (CAUSAL) causal_groups(a.num_units / ((a.num_q_tiles + 1) / 2), a.N, D, sms, &args.group_big,
+                            &args.num_big_groups);
+  SchedPool& pool = g_sched_pool[dev];
+  std::unique_lock<std::mutex> lock(pool.mu, std::defer_lock);
+  int slot = -1;
+  if (CAUSAL && ctas > 1) {
+    lock.lock();
+    slot = sched_slot(pool, st);
+    if (slot >= 0) args.sched = pool.base + 2 * slot;
+  }
+  kern<<<dim3((unsigned)ctas), 384, smem, st>>>(mq, mk, mv, args);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "fattn_fwd_kernel launch");
+  if (e != cudaSuccess && e != cudaErrorNotReady) return cuda_fail(e, "fattn_fwd_kernel launch");
+  if (slot >= 0) {
+    e = cudaEventRecord(pool.ev[slot], st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
   return FATTN_OK;
 }
 
@@ -257,23 +375,24 @@ int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, 
     return FATTN_ERR_ALIGNMENT;
 
   const uint64_t rows = (uint64_t)B * H * N;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv;
   if (int rc = make_bf16_tile_map(&mq, q, rows, d)) return rc;
   if (int rc = make_bf16_tile_map(&mk, k, rows, d)) return rc;
   if (int rc = make_bf16_tile_map(&mv, v, rows, d)) return rc;
-  if (int rc = make_bf16_tile_map(&mo, o, rows, d)) return rc;
 
   fattn::FwdArgs a;
   a.lse = lse;
+  a.o = static_cast<__nv_bfloat16*>(o);
   a.N = N;
   a.num_q_tiles = N / 128;
+  a.num_units = B * H * ((N / 128 + 1) / 2);
+  a.group_big = 1;
+  a.num_big_groups = 1;
+  a.sched = nullptr;
   a.scale_log2 = scale * kLog2e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, mo, a, BH, st)
-                             : launch_fwd<64, false>(mq, mk, mv, mo, a, BH, st);
-  return causal ? launch_fwd<128, true>(mq, mk, mv, mo, a, BH, st)
-                : launch_fwd<128, false>(mq, mk, mv, mo, a, BH, st);
+  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, a, st) : launch_fwd<64, false>(mq, mk, mv, a, st);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, a, st) : launch_fwd<128, false>(mq, mk, mv, a, st);
 }
 
 int fattn_exp2_poly(const float* x, float* y, long long n, fattn_stream_t stream) {

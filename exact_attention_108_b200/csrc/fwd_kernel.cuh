@@ -1,22 +1,26 @@
 // fwd_kernel.cuh -- fused exact-attention forward for sm_100a.
 //
-// One CTA owns two consecutive 128-row query tiles of one (batch, head).  It
-// streams the 128-row key/value tiles of that head through a shared-memory ring
-// and keeps the running row max m and row sum l of the online softmax in
-// registers, so the N x N score matrix never leaves the chip (page 2 "一、用分块
+// A persistent CTA (one per SM) loops over work units, each two consecutive
+// 128-row query tiles of one (batch, head).  It streams the 128-row key/value
+// tiles of that head through a shared-memory ring and keeps the running row max
+// m and row sum l of the online softmax in registers, so the N x N score matrix
+// never leaves the chip (page 2 "一、用分块
 // 计算提高片上数据复用" and "二、在线 Softmax 保持精确结果"; page 3 "4.1 分块计算"
 // and "4.2 在线softmax技巧").  Only O and the per-row log-sum-exp are written
 // (page 2 "三、融合算子减少中间张量落盘").
 //
 // Roles (384 threads = three warpgroups, warp-specialised):
-//   warps 0..3  softmax group 0, thread = row of query tile 0   (224 registers)
-//   warps 4..7  softmax group 1, thread = row of query tile 1   (224 registers)
-//   warp 8      TMA producer: Q0, Q1 once, then K_j, V_j through an NSLOT-deep ring
-//   warp 9      tcgen05 issuer (one thread); warps 10, 11 idle   (56 registers)
+//   warps 0..3  softmax group 0, thread = row of query tile 0   (208 registers)
+//   warps 4..7  softmax group 1, thread = row of query tile 1   (208 registers)
+//   warp 8      TMA producer: Q tiles through a 3-buffer ring, K_j, V_j through
+//               an NSLOT-deep ring; it also hands the work units to the others
+//   warp 9      tcgen05 issuer (one thread); warps 10, 11 idle   (88 registers)
 //                 S0 = Q0 K_j^T, S1 = Q1 K_j^T          (TMEM, fp32)
 //                 O0 += P0 V_j,  O1 += P1 V_j           (P read from TMEM)
 // While group 0 turns S0 into P0 the tensor cores compute S1 (and vice versa),
-// so the exponentials of one tile overlap the products of the other.
+// so the exponentials of one tile overlap the products of the other.  The Q
+// ring has a third buffer, so the next unit's first query tile loads while the
+// current unit still holds two.
 //
 // Tensor memory (512 columns x 128 lanes): S0 at column 0, S1 at 128 (P_k, bf16,
 // overlays the first 64 columns of S_k), O0 at 256, O1 at 256 + D.
@@ -34,10 +38,19 @@
 namespace fattn {
 
 struct FwdArgs {
-  float* lse;         // [B*H*N] fp32
-  int N;              // keys per head (multiple of 128)
-  int num_q_tiles;    // N / 128
-  float scale_log2;   // scale * log2(e)
+  float* lse;            // [B*H*N] fp32
+  __nv_bfloat16* o;      // [B*H*N, D] bf16
+  int N;                 // keys per head (multiple of 128)
+  int num_q_tiles;       // N / 128
+  int num_units;         // B*H * ceil(num_q_tiles / 2)
+  int group_big;         // causal order: heads in each of the first num_big_groups groups;
+  int num_big_groups;    //   the remaining groups hold group_big - 1 heads
+  // Causal only, may be null: two device counters (next unit ticket, CTAs
+  // finished), both 0 at launch and returned to 0 by the last CTA.  With them
+  // each CTA claims its next unit when it runs short of work; without them CTA c
+  // takes units c, c + gridDim.x, ...
+  unsigned int* sched;
+  float scale_log2;      // scale * log2(e)
 };
 
 template <int D>
@@ -45,14 +58,22 @@ struct FwdCfg {
   static constexpr int KB = D / 64;                 // 128-byte column blocks per row
   static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row Q/K/V tile
   static constexpr int BLK = 128 * 128;             // one 64-column block of a tile
+  static constexpr int QBUF = 3;                    // Q tile ring
   static constexpr int NSLOT = (D == 128) ? 4 : 6;  // K/V ring depth
-  static constexpr int OFF_Q = 0;                   // Q0, Q1 (reused for the O epilogue)
-  static constexpr int OFF_SLOT = 2 * TILE;
+  static constexpr int NUNIT = 4;                   // ring of unit indices from the producer
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_SLOT = QBUF * TILE;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * TILE;
-  // q_full, slot_full[NSLOT], slot_empty[NSLOT], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int NBAR = 1 + 2 * NSLOT + 6 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (4 B), abort flag (4 B)
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;    // + slack for 1024-byte alignment
+  // barriers: q_full[QBUF], q_empty[QBUF], slot_full[NSLOT], slot_empty[NSLOT],
+  // s_full[2], p_full[2], pv_done[2], o_free[2], drain, unit_full[NUNIT], unit_empty[NUNIT]
+  static constexpr int B_QF = 0, B_QE = QBUF, B_SF = 2 * QBUF, B_SE = B_SF + NSLOT;
+  static constexpr int B_S = B_SE + NSLOT, B_P = B_S + 2, B_PV = B_S + 4, B_OF = B_S + 6;
+  static constexpr int B_DRAIN = B_S + 8, B_UF = B_DRAIN + 1, B_UE = B_UF + NUNIT;
+  static constexpr int NBAR = B_UE + NUNIT;
+  // tmem base (4 B), abort flag (4 B), pad (8 B), unit ring (4 B each)
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 4 * NUNIT + 1024;  // + slack for 1024-byte alignment
+  static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr int TMEM_COLS = 512;
   static constexpr int TM_S = 0;                       // S_k at k * 128
   static constexpr int TM_O = 256;                     // O_k at 256 + k * D
@@ -73,53 +94,91 @@ enum : int {  // wait sites recorded in the device status word on a timeout
   kSiteFwdMmaV = 0x106,
   kSiteFwdSoftS = 0x107,
   kSiteFwdSoftO = 0x108,
+  kSiteFwdMmaO = 0x109,
+  kSiteFwdUnit = 0x10a,
 };
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                     const FwdArgs args) {
+                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
   using C = FwdCfg<D>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
 
-  auto sQ = [&](int k) { return sbase + C::OFF_Q + k * C::TILE; };
+  auto sQ = [&](int b) { return sbase + C::OFF_Q + b * C::TILE; };
   const uint32_t sSlot0 = sbase + C::OFF_SLOT;
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t bar_q_full = bar0;
-  auto bar_slot_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto bar_slot_empty = [&](int s) { return bar0 + 8u * (1 + C::NSLOT + s); };
-  auto bar_s_full = [&](int k) { return bar0 + 8u * (1 + 2 * C::NSLOT + k); };
-  auto bar_p_full = [&](int k) { return bar0 + 8u * (3 + 2 * C::NSLOT + k); };
-  auto bar_pv_done = [&](int k) { return bar0 + 8u * (5 + 2 * C::NSLOT + k); };
-  const uint32_t bar_drain = bar0 + 8u * (7 + 2 * C::NSLOT);
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  auto bar_q_full = [&](int b) { return bar(C::B_QF + b); };
+  auto bar_q_empty = [&](int b) { return bar(C::B_QE + b); };
+  auto bar_slot_full = [&](int s) { return bar(C::B_SF + s); };
+  auto bar_slot_empty = [&](int s) { return bar(C::B_SE + s); };
+  auto bar_s_full = [&](int k) { return bar(C::B_S + k); };
+  auto bar_p_full = [&](int k) { return bar(C::B_P + k); };
+  auto bar_pv_done = [&](int k) { return bar(C::B_PV + k); };
+  auto bar_o_free = [&](int k) { return bar(C::B_OF + k); };
+  const uint32_t bar_drain = bar(C::B_DRAIN);
+  auto bar_unit_full = [&](int e) { return bar(C::B_UF + e); };
+  auto bar_unit_empty = [&](int e) { return bar(C::B_UE + e); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: a pair of query tiles; the pair index varies fastest so that the
-  // CTAs resident at one time share a head's K/V in L2.  Causal heads start with
-  // their longest pairs.
+  // Work units.  Non-causal heads: batch*head slowest, then the pair of query
+  // tiles; every unit costs the same.  Causal heads: the heads form groups of
+  // group_big or group_big - 1; inside a group the longest pairs of all its heads
+  // come first (longest-processing-time order), so the group's short units fill
+  // in behind its long ones, while the group's keys and values stay in L2.
   const int NT = args.num_q_tiles;
   const int NP = (NT + 1) >> 1;
-  const int bh = (int)(blockIdx.x / (unsigned)NP);
-  const int p_in_head = (int)(blockIdx.x % (unsigned)NP);
-  const int pair = CAUSAL ? (NP - 1 - p_in_head) : p_in_head;
-  const int head_row0 = bh * args.N;
-  const int tile0 = 2 * pair;
-  const bool has_q1 = tile0 + 1 < NT;
-  // key tiles each query tile needs (contiguous from 0)
-  const int n_kv0 = CAUSAL ? tile0 + 1 : NT;
-  const int n_kv1 = has_q1 ? (CAUSAL ? tile0 + 2 : NT) : 0;
-  const int n_kv = n_kv1 > n_kv0 ? n_kv1 : n_kv0;
+  const bool dyn = CAUSAL && args.sched != nullptr;
+  struct Unit {
+    int head_row0, tile0, n_kv0, n_kv1, n_kv;
+  };
+  auto unit_of = [&](int u) {
+    Unit w;
+    int bh, pair;
+    if (CAUSAL) {
+      const int big = args.group_big, ubig = NP * big, nbig_units = args.num_big_groups * ubig;
+      int r, hg, h0;
+      if (u < nbig_units) {
+        const int g = u / ubig;
+        r = u - g * ubig;
+        hg = big;
+        h0 = g * big;
+      } else {
+        const int gs = NP * (big - 1), u2 = u - nbig_units, g = u2 / gs;
+        r = u2 - g * gs;
+        hg = big - 1;
+        h0 = args.num_big_groups * big + g * (big - 1);
+      }
+      bh = h0 + r % hg;
+      pair = NP - 1 - r / hg;
+    } else {
+      bh = u / NP;
+      pair = u % NP;
+    }
+    w.head_row0 = bh * args.N;
+    w.tile0 = 2 * pair;
+    const bool has_q1 = w.tile0 + 1 < NT;
+    // key tiles each query tile needs (contiguous from 0); 0 = tile absent
+    w.n_kv0 = CAUSAL ? w.tile0 + 1 : NT;
+    w.n_kv1 = has_q1 ? (CAUSAL ? w.tile0 + 2 : NT) : 0;
+    w.n_kv = w.n_kv1 > w.n_kv0 ? w.n_kv1 : w.n_kv0;
+    return w;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q_full, 1);
+    for (int b = 0; b < C::QBUF; ++b) {
+      mbar_init(bar_q_full(b), 1);
+      mbar_init(bar_q_empty(b), 1);
+    }
     for (int s = 0; s < C::NSLOT; ++s) {
       mbar_init(bar_slot_full(s), 1);
       mbar_init(bar_slot_empty(s), 1);
@@ -128,8 +187,13 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar_s_full(k), 1);
       mbar_init(bar_p_full(k), 128);
       mbar_init(bar_pv_done(k), 1);
+      mbar_init(bar_o_free(k), 128);
     }
     mbar_init(bar_drain, 1);
+    for (int e = 0; e < C::NUNIT; ++e) {
+      mbar_init(bar_unit_full(e), 1);
+      mbar_init(bar_unit_empty(e), 1 + 8);  // the MMA thread and one lane of each softmax warp
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -143,40 +207,63 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   // 384 threads launch with 168 registers each (64512 in all); the softmax groups
-  // take 224, the producer/MMA group keeps 56: 2*128*224 + 128*56 = 64512.
+  // take 208, the producer/MMA group keeps 88: 2*128*208 + 128*88 = 64512.
   if (warp >= 8) {
-    regs_decrease<56>();
+    regs_decrease<88>();
     if (warp == 8) {
       // ------------------------------------------------------------ producer
       if (lane == 0) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_o);
-        mbar_arrive_expect_tx(bar_q_full, (has_q1 ? 2 : 1) * C::TILE);
-        for (int k = 0; k < (has_q1 ? 2 : 1); ++k)
-  #pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_2d(sQ(k) + kb * C::BLK, &tm_q, bar_q_full, kb * 64, head_row0 + (tile0 + k) * 128);
-        int it = 0;
+        int it = 0;  // K/V tiles loaded (ring position), continuous across units
+        int qs = 0;  // Q tiles loaded (Q ring position)
         bool ok = true;
-        for (int j = 0; j < n_kv && ok; ++j) {
-          for (int t = 0; t < 2; ++t, ++it) {
-            const int s = it % C::NSLOT;
-            if (!mbar_wait(bar_slot_empty(s), ((it / C::NSLOT) & 1) ^ 1, abort_flag, kSiteFwdProducer)) {
-              ok = false;
-              break;
+        int u = blockIdx.x;  // the first unit by block index
+        for (int nu = 0; ok; ++nu) {
+          const int e = nu % C::NUNIT;
+          if (!(ok = mbar_wait(bar_unit_empty(e), ((nu / C::NUNIT) & 1) ^ 1, abort_flag, kSiteFwdUnit))) break;
+          unit_ring[e] = u < args.num_units ? u : -1;
+          mbar_arrive(bar_unit_full(e));
+          if (u >= args.num_units) break;
+          const Unit w = unit_of(u);
+          const int nq = w.n_kv1 > 0 ? 2 : 1;
+          unsigned int ticket = 0;
+          for (int j = 0; j < w.n_kv && ok; ++j) {
+            // A dynamic CTA claims its next unit as the loads of this unit's last
+            // key/value tile go out: late enough that no CTA sits on a unit while
+            // another has run out of work, early enough to hide the atomic.
+            if (dyn && j == w.n_kv - 1) ticket = atomicAdd(args.sched, 1u);
+            for (int t = 0; t < 2 && ok; ++t) {
+              const int s = it % C::NSLOT;
+              if (!(ok = mbar_wait(bar_slot_empty(s), ((it / C::NSLOT) & 1) ^ 1, abort_flag, kSiteFwdProducer)))
+                break;
+              mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
+              const CUtensorMap* map = (t == 0) ? &tm_k : &tm_v;
+              const uint32_t dst = sSlot0 + s * C::TILE;
+#pragma unroll
+              for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_2d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, w.head_row0 + j * 128);
+              ++it;
+              // Q0 after K_0, Q1 after V_0: each into the Q buffer freed longest ago
+              if (j == 0 && t < nq) {
+                const int b = qs % C::QBUF;
+                if (!(ok = mbar_wait(bar_q_empty(b), ((qs / C::QBUF) & 1) ^ 1, abort_flag, kSiteFwdProducer)))
+                  break;
+                mbar_arrive_expect_tx(bar_q_full(b), C::TILE);
+#pragma unroll
+                for (int kb = 0; kb < C::KB; ++kb)
+                  tma_load_2d(sQ(b) + kb * C::BLK, &tm_q, bar_q_full(b), kb * 64,
+                              w.head_row0 + (w.tile0 + t) * 128);
+                ++qs;
+              }
             }
-            mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
-            const CUtensorMap* map = (t == 0) ? &tm_k : &tm_v;
-            const uint32_t dst = sSlot0 + s * C::TILE;
-  #pragma unroll
-            for (int kb = 0; kb < C::KB; ++kb)
-              tma_load_2d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, head_row0 + j * 128);
           }
+          u = dyn ? (int)gridDim.x + (int)ticket : u + (int)gridDim.x;
         }
         if (!ok) {  // aborted: let the copies already issued land before the CTA exits
-          mbar_wait_ns(bar_q_full, 0, 100000000ull);
+          for (int i = (qs > C::QBUF ? qs - C::QBUF : 0); i < qs; ++i)
+            mbar_wait_ns(bar_q_full(i % C::QBUF), (i / C::QBUF) & 1, 100000000ull);
           for (int i = (it > C::NSLOT ? it - C::NSLOT : 0); i < it; ++i)
             mbar_wait_ns(bar_slot_full(i % C::NSLOT), (i / C::NSLOT) & 1, 100000000ull);
         }
@@ -187,53 +274,89 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
         constexpr uint32_t idPV = idesc_bf16_f32(128, D, false, true);    // P (TMEM) x V (MN-major)
-        bool ok = mbar_wait(bar_q_full, 0, abort_flag, kSiteFwdMmaQ);
-        auto act = [&](int k, int j) { return j < (k == 0 ? n_kv0 : n_kv1); };
-        auto slot_of = [&](int it) { return it % C::NSLOT; };
-        auto issue_s = [&](int k, int j) {  // S_k = Q_k K_j^T
-          const uint32_t kaddr = sSlot0 + slot_of(2 * j) * C::TILE;
+        auto slot_of = [&](int i) { return i % C::NSLOT; };
+        auto issue_s = [&](int k, int qbuf, int kslot) {  // S_k = Q K^T, Q from buffer qbuf, K from ring slot kslot
+          // The start address is a descriptor's low 14 bits (address / 16, below
+          // 2^14 for any shared-memory address), so each K step adds a constant to
+          // one base descriptor per operand.  The bases pass through an opaque
+          // move: hoisted out of the loops, the descriptors of every buffer and
+          // step would not fit in this thread's registers.
+          const uint64_t dq = sdesc_sw128(opaque_u32(sQ(qbuf)), 16);
+          const uint64_t dk = sdesc_sw128(opaque_u32(sSlot0 + kslot * C::TILE), 16);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(tmem + C::TM_S + k * 128, sdesc_sw128(sQ(k) + off, 16), sdesc_sw128(kaddr + off, 16), idS,
-                   kk > 0 ? 1u : 0u);
+            const uint32_t off16 = ((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + C::TM_S + k * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_s_full(k));
         };
-        // Issue order: S0_0 S1_0 | PV0_0 S0_1 | PV1_0 S1_1 | PV0_1 S0_2 | ...  While one
-        // softmax group works on S_k, the tensor cores run the other group's P V and
-        // its next S.  S_k(j+1) overwrites the columns PV_k(j) reads P_k(j) from; the
-        // tcgen05.mma instructions of one thread execute in issue order.
-        if (ok) ok = mbar_wait(bar_slot_full(slot_of(0)), 0, abort_flag, kSiteFwdMmaK);
-        if (ok) {
-          tc_fence_after();
-          for (int k = 0; k < 2; ++k)
-            if (act(k, 0)) issue_s(k, 0);
-          mma_commit(bar_slot_empty(slot_of(0)));
-        }
-        for (int j = 0; j < n_kv && ok; ++j) {
-          const int itV = 2 * j + 1, itK1 = 2 * j + 2;
-          if (!(ok = mbar_wait(bar_slot_full(slot_of(itV)), (itV / C::NSLOT) & 1, abort_flag, kSiteFwdMmaV))) break;
-          const bool more = j + 1 < n_kv;
-          if (more &&
-              !(ok = mbar_wait(bar_slot_full(slot_of(itK1)), (itK1 / C::NSLOT) & 1, abort_flag, kSiteFwdMmaK)))
-            break;
-          const uint32_t vaddr = sSlot0 + slot_of(itV) * C::TILE;
-          for (int k = 0; k < 2; ++k) {
-            if (!act(k, j)) continue;
-            if (!(ok = mbar_wait(bar_p_full(k), j & 1, abort_flag, kSiteFwdMmaP))) break;
+        int it = 0;          // ring position of the current unit's K_0
+        int qs = 0;          // Q ring position of the current unit's Q0
+        int tk[2] = {0, 0};  // tiles processed per query-tile slot (phases of s_full/p_full/pv_done)
+        int uk[2] = {0, 0};  // units in which each query-tile slot was active (phases of o_free)
+        bool ok = true;
+        for (int nu = 0; ok; ++nu) {
+          const int e = nu % C::NUNIT;
+          if (!(ok = mbar_wait(bar_unit_full(e), (nu / C::NUNIT) & 1, abort_flag, kSiteFwdUnit))) break;
+          const int u = unit_ring[e];
+          mbar_arrive(bar_unit_empty(e));
+          if (u < 0) break;
+          const Unit w = unit_of(u);
+          const int nq = w.n_kv1 > 0 ? 2 : 1;
+          const int it0 = it;
+          auto n_kv_of = [&](int k) { return k == 0 ? w.n_kv0 : w.n_kv1; };
+          auto qbuf = [&](int k) { return (qs + k) % C::QBUF; };
+          // prologue: S_k(0).  S_k(0) of a unit overwrites the columns the previous
+          // unit's last PV_k read P_k from; tcgen05.mma of one thread execute in
+          // issue order.
+          if (!(ok = mbar_wait(bar_slot_full(slot_of(it0)), (it0 / C::NSLOT) & 1, abort_flag, kSiteFwdMmaK))) break;
+          for (int k = 0; k < nq && ok; ++k) {
+            if (!(ok = mbar_wait(bar_q_full(qbuf(k)), ((qs + k) / C::QBUF) & 1, abort_flag, kSiteFwdMmaQ))) break;
             tc_fence_after();
-            const uint32_t tP = tmem + C::TM_S + k * 128;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step = 8 TMEM columns of packed P
-              mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, sdesc_sw128(vaddr + kk * 2048, C::BLK), idPV,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(bar_pv_done(k));
-            if (more && act(k, j + 1)) issue_s(k, j + 1);
+            issue_s(k, qbuf(k), slot_of(it0));
+            if (n_kv_of(k) == 1) mma_commit(bar_q_empty(qbuf(k)));  // Q_k's only product
           }
           if (!ok) break;
-          mma_commit(bar_slot_empty(slot_of(itV)));
-          if (more) mma_commit(bar_slot_empty(slot_of(itK1)));
+          mma_commit(bar_slot_empty(slot_of(it0)));
+          // Issue order: S0_0 S1_0 | PV0_0 S0_1 | PV1_0 S1_1 | PV0_1 S0_2 | ...  While one
+          // softmax group works on S_k, the tensor cores run the other group's P V and
+          // its next S.  S_k(j+1) overwrites the columns PV_k(j) reads P_k(j) from.
+          for (int j = 0; j < w.n_kv && ok; ++j) {
+            const int itV = it0 + 2 * j + 1, itK1 = it0 + 2 * j + 2;
+            if (!(ok = mbar_wait(bar_slot_full(slot_of(itV)), (itV / C::NSLOT) & 1, abort_flag, kSiteFwdMmaV)))
+              break;
+            const bool more = j + 1 < w.n_kv;
+            if (more &&
+                !(ok = mbar_wait(bar_slot_full(slot_of(itK1)), (itK1 / C::NSLOT) & 1, abort_flag, kSiteFwdMmaK)))
+              break;
+            const uint32_t vaddr = sSlot0 + slot_of(itV) * C::TILE;
+            for (int k = 0; k < 2 && ok; ++k) {
+              if (j >= n_kv_of(k)) continue;
+              // the first P V of a unit overwrites O_k: the previous epilogue must have read it
+              if (j == 0 && uk[k] > 0 &&
+                  !(ok = mbar_wait(bar_o_free(k), (uk[k] - 1) & 1, abort_flag, kSiteFwdMmaO)))
+                break;
+              if (!(ok = mbar_wait(bar_p_full(k), tk[k] & 1, abort_flag, kSiteFwdMmaP))) break;
+              tc_fence_after();
+              const uint32_t tP = tmem + C::TM_S + k * 128;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step = 8 TMEM columns of packed P
+                mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, sdesc_sw128(vaddr + kk * 2048, C::BLK), idPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(bar_pv_done(k));
+              ++tk[k];
+              if (j + 1 < n_kv_of(k)) {
+                issue_s(k, qbuf(k), slot_of(itK1));
+                if (j + 2 == n_kv_of(k)) mma_commit(bar_q_empty(qbuf(k)));  // Q_k's last product
+              }
+            }
+            if (!ok) break;
+            mma_commit(bar_slot_empty(slot_of(itV)));
+            if (more) mma_commit(bar_slot_empty(slot_of(itK1)));
+          }
+          it = it0 + 2 * w.n_kv;
+          qs += nq;
+          for (int k = 0; k < nq; ++k) ++uk[k];
         }
         // Make sure nothing this thread issued is still running before TMEM is freed.
         mma_commit(bar_drain);
@@ -242,150 +365,154 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     }
   } else {
-    regs_increase<224>();
+    regs_increase<208>();
     // ------------------------------------------------------ softmax groups
-    const int k = warp >> 2;  // query tile of this group
+    const int k = warp >> 2;  // query-tile slot of this group
     const int wq = warp & 3;
     const int r = wq * 32 + lane;  // row inside the query tile
-    const int n_kv_k = k == 0 ? n_kv0 : n_kv1;
-    const int q_tile = tile0 + k;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + C::TM_S + k * 128 + lane_off;
     const uint32_t tO = tmem + C::TM_O + k * D + lane_off;
     const float sl2 = args.scale_log2;
-    float m_ref = -INFINITY;  // reference max of the scaled scores, log2 units
-    float l = 0.f;            // running sum of exp2(score - m_ref)
+    int tk = 0;  // tiles processed (phases of s_full/p_full/pv_done for this slot)
     bool ok = true;
-    for (int j = 0; j < n_kv_k; ++j) {
-      ok = mbar_wait(bar_s_full(k), j & 1, abort_flag, kSiteFwdSoftS);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      tc_fence_after();
-      uint32_t v[4][32];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, v[c4]);
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld_wait(v[c4]);
-      if (CAUSAL && j == q_tile) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > r) v[c >> 5][c & 31] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
-      }
-      // row max of the raw scores, turned into the max of scale * score (log2 units);
-      // four independent three-input chains keep the dependencies short
-      float mx;
-      {
-        float pm[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) pm[u] = __uint_as_float(v[u][0]);
-        if (sl2 >= 0.f) {
-#pragma unroll
-          for (int c = 0; c < 128; c += 8)
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
-                            __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
-          mx = fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; c += 8)
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
-                            __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
-          mx = fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
-        }
-        mx *= sl2;
-      }
-      // lazily move the reference max; rescale O and l only when it moves
-      const bool grow = mx > m_ref + kRescaleThreshold;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float m_new = fmaxf(m_ref, mx);
-        const float alpha = ex2(m_ref - m_new);  // 0 on the first tile (m_ref = -inf)
-        l *= alpha;
-        m_ref = m_new;
-        if (j > 0) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_ld_wait(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-      }
-      const bool diag = CAUSAL && j == q_tile;  // keys c > r of this tile are masked
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
-      uint32_t pk[2][32];                          // P row as packed bf16 pairs
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
-                                           __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
-                                   sl2x2, negm2);
-        float p0, p1;
-        if (((c >> 1) & 7) < kPolyPairsPer8) {
-          f2_unpack(exp2_poly_x2(x2), p0, p1);  // on the FMA pipe
-        } else {
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          p0 = ex2(x0);
-          p1 = ex2(x1);
-        }
-        if (diag) {
-          p0 = (c > r) ? 0.f : p0;
-          p1 = (c + 1 > r) ? 0.f : p1;
-        }
-        acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
-        pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
-      }
-      {
-        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-        float s0, s1;
-        f2_unpack(a2, s0, s1);
-        l += s0 + s1;
-      }
-      // P (bf16 pairs) over the first 64 columns of S_k
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_p_full(k));
-    }
-    if (ok && n_kv_k > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done(k), (n_kv_k - 1) & 1, abort_flag, kSiteFwdSoftO));
-      if (ok) {
+    for (int nu = 0; ok; ++nu) {
+      const int e = nu % C::NUNIT;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_unit_full(e), (nu / C::NUNIT) & 1, abort_flag, kSiteFwdUnit));
+      if (!ok) break;
+      const int u = unit_ring[e];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_unit_empty(e));
+      if (u < 0) break;
+      const Unit w = unit_of(u);
+      const int n_kv_k = k == 0 ? w.n_kv0 : w.n_kv1;
+      if (n_kv_k == 0) continue;  // no second query tile in this unit
+      const int q_tile = w.tile0 + k;
+      float m_ref = -INFINITY;  // reference max of the scaled scores, log2 units
+      float l = 0.f;            // running sum of exp2(score - m_ref)
+      for (int j = 0; j < n_kv_k; ++j, ++tk) {
+        ok = mbar_wait(bar_s_full(k), tk & 1, abort_flag, kSiteFwdSoftS);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
-        const float inv_l = 1.f / l;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_ld_wait(o);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = (c & 1) * 4 + q4;
-            const uint32_t* w = &o[q4 * 8];
-            st_shared_v4(sQ(k) + (c >> 1) * C::BLK + sw128_offset(r, chunk),
-                         pack_bf16x2(__uint_as_float(w[0]) * inv_l, __uint_as_float(w[1]) * inv_l),
-                         pack_bf16x2(__uint_as_float(w[2]) * inv_l, __uint_as_float(w[3]) * inv_l),
-                         pack_bf16x2(__uint_as_float(w[4]) * inv_l, __uint_as_float(w[5]) * inv_l),
-                         pack_bf16x2(__uint_as_float(w[6]) * inv_l, __uint_as_float(w[7]) * inv_l));
+        uint32_t v[4][32];
+  #pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, v[c4]);
+  #pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld_wait(v[c4]);
+        if (CAUSAL && j == q_tile) {
+  #pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > r) v[c >> 5][c & 31] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
+        }
+        // row max of the raw scores, turned into the max of scale * score (log2 units);
+        // four independent three-input chains keep the dependencies short
+        float mx;
+        {
+          float pm[4];
+  #pragma unroll
+          for (int u = 0; u < 4; ++u) pm[u] = __uint_as_float(v[u][0]);
+          if (sl2 >= 0.f) {
+  #pragma unroll
+            for (int c = 0; c < 128; c += 8)
+  #pragma unroll
+              for (int u = 0; u < 4; ++u)
+                pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                              __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+            mx = fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3]));
+          } else {
+  #pragma unroll
+            for (int c = 0; c < 128; c += 8)
+  #pragma unroll
+              for (int u = 0; u < 4; ++u)
+                pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                              __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+            mx = fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
+          }
+          mx *= sl2;
+        }
+        // lazily move the reference max; rescale O and l only when it moves
+        const bool grow = mx > m_ref + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float m_new = fmaxf(m_ref, mx);
+          const float alpha = ex2(m_ref - m_new);  // 0 on the first tile (m_ref = -inf)
+          l *= alpha;
+          m_ref = m_new;
+          if (j > 0) {
+  #pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_ld_wait(o);
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(tO + c * 32, o);
+            }
           }
         }
-        // natural-log LSE of the scaled scores: (m_ref + log2 l) * ln 2
-        args.lse[head_row0 + q_tile * 128 + r] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
-        fence_async_shared();
-        named_barrier(1 + k, 128);
-        if (r == 0) {
-#pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_store_2d(&tm_o, sQ(k) + kb * C::BLK, kb * 64, head_row0 + q_tile * 128);
-          bulk_commit();
-          bulk_wait0();
+        const bool diag = CAUSAL && j == q_tile;  // keys c > r of this tile are masked
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
+        uint32_t pk[2][32];                          // P row as packed bf16 pairs
+  #pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
+                                             __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
+                                     sl2x2, negm2);
+          float p0, p1;
+          if (((c >> 1) & 7) < kPolyPairsPer8) {
+            f2_unpack(exp2_poly_x2(x2), p0, p1);  // on the FMA pipe
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          if (diag) {
+            p0 = (c > r) ? 0.f : p0;
+            p1 = (c + 1 > r) ? 0.f : p1;
+          }
+          acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
+          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
         }
+        {
+          const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float s0, s1;
+          f2_unpack(a2, s0, s1);
+          l += s0 + s1;
+        }
+        // P (bf16 pairs) over the first 64 columns of S_k
+        tmem_st32(tS, pk[0]);
+        tmem_st32(tS + 32, pk[1]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(k));
       }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done(k), (tk - 1) & 1, abort_flag, kSiteFwdSoftO));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t o[D / 32][32];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld_wait(o[c]);
+      tc_fence_before();
+      mbar_arrive(bar_o_free(k));  // O_k may now be overwritten by the next unit
+      // O row (bf16) straight to global memory, LSE (natural log) beside it
+      const float inv_l = 1.f / l;
+      const size_t row = (size_t)(w.head_row0 + q_tile * 128 + r);
+      uint4* dst = reinterpret_cast<uint4*>(args.o + row * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t* x = &o[c][q4 * 8];
+          dst[c * 4 + q4] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
+        }
+      args.lse[row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
     }
     tc_fence_before();
   }
@@ -393,6 +520,15 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (dyn && threadIdx.x == 0) {
+    // the last CTA to finish returns both counters to 0 for the next launch
+    __threadfence();
+    if (atomicAdd(args.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(args.sched, 0u);
+      atomicExch(args.sched + 1, 0u);
+      __threadfence();
+    }
   }
 }
 

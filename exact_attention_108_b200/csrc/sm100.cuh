@@ -217,6 +217,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 // K-major: rows of 128 bytes (64 bf16 along K), 8-row groups SBO = 1024 bytes apart; LBO unused.
 // MN-major: 64 MN-contiguous elements per 128-byte row, K rows 128 bytes apart, 8-row groups
 //   SBO = 1024 bytes apart, next 64-element MN chunk LBO bytes further.
+// x, through a volatile move the compiler cannot look through: values derived
+// from it are computed where they are used instead of hoisted out of loops.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+  uint32_t y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);

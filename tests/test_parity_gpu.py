@@ -59,11 +59,12 @@ def test_tiny_workload_forward_backward():
 
 def _check_o_derived(o, o_ref, v_ref):
     """Off-workload scales: the bound the arithmetic itself gives.  P is rounded
-    to bf16 before the PV product (relative error <= 2^-9 per weight, so at most
-    2^-9 * max|V| on a row) and O is rounded to bf16 on output (<= 2^-9 |O|);
-    the bound doubles both for the fp32 accumulation and exp2 approximation."""
+    to bf16 before the PV product (unit roundoff 2^-8 per weight, so at most
+    2^-8 * max|V| on a row) and O is rounded to bf16 on output (<= 2^-8 |O|).
+    The fp32 exponentials and accumulation add errors near 2^-20 relative per
+    term, covered by a 2^-14 * max|V| allowance."""
     err = np.abs(to_f64(o) - o_ref)
-    bound = 2.0 ** -8 * (np.abs(v_ref).max() + np.abs(o_ref))
+    bound = 2.0 ** -8 * (np.abs(v_ref).max() + np.abs(o_ref)) + 2.0 ** -14 * np.abs(v_ref).max()
     assert (err <= bound).all(), f"O error {err.max():.3e} exceeds the bf16 rounding bound"
     assert err.mean() <= 1e-3
 
