@@ -30,10 +30,13 @@
  * B * H * N < 2^31.  scale must be finite (any sign).
  *
  * Ownership and asynchrony.  The caller allocates and owns every buffer,
- * including the backward workspace.  The library allocates no device memory
- * and keeps no per-call state.  Every call only enqueues work on `stream` and
- * returns; results are valid once the stream has been synchronised.  Inputs
- * must stay alive until then.
+ * including the backward workspace.  The library allocates no device memory at
+ * run time.  Its only device state is static: 16 pairs of scheduling counters
+ * for the causal forward, and the scratch array of fattn_bwd_noalloc.  It also
+ * keeps 16 CUDA events per device, created by the first causal forward on that
+ * device.  Every call only enqueues work on `stream` and returns; results are
+ * valid once the stream has been synchronised.  Inputs must stay alive until
+ * then.
  *
  * Errors.  Arguments are validated before anything is enqueued; an invalid
  * call returns a non-zero status and has no side effects.  A failed launch
@@ -70,6 +73,13 @@ typedef enum {
  *   q, k, v : inputs, read only.
  *   causal  : 0 = no mask, 1 = query i attends keys 0..i.
  *   scale   : multiplies QK^T (usually 1/sqrt(d)).
+ * One CTA per SM loops over units of two 128-row query tiles.  A causal launch
+ * lets its CTAs claim units from one of the static counter pairs.  It takes a
+ * pair only when the event recorded after that pair's previous launch has
+ * completed; that launch returned the pair to zero.  A launch during stream
+ * capture, or one that finds every pair busy, assigns units round-robin.  The
+ * schedule does not change the results: every unit is computed the same way,
+ * whichever CTA takes it.
  */
 int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
               int B, int H, int N, int d, int causal, float scale,
