@@ -88,6 +88,8 @@ struct BwdArgs {
   float* dq_acc;      // [B*H*N, D] fp32
   int N;
   int num_tiles;      // N / 128
+  int group_big;      // causal order: heads in each of the first num_big_groups groups;
+  int num_big_groups; //   the remaining groups hold group_big - 1 heads
   float scale;        // for dK
   float scale_log2;   // scale * log2(e)
 };
@@ -172,11 +174,34 @@ __global__ void __launch_bounds__(384, 1)
     return;
   }
   const int NT = args.num_tiles;
-  // The key tile varies fastest so that the CTAs resident at one time add into
-  // the same head's dQ rows (which then stay in L2); causal: tile 0 sees the most
-  // query tiles and is launched first.
-  const int bh = (int)(blockIdx.x / (unsigned)NT);
-  const int kv_tile = (int)(blockIdx.x % (unsigned)NT);
+  // Non-causal: the key tile varies fastest, so the CTAs resident at one time add
+  // into the same head's dQ rows (which then stay in L2).  Causal: a key tile's
+  // work falls with its index (tile t sees NT - t query tiles), so the heads form
+  // groups of group_big or group_big - 1 and inside a group the longest tiles of
+  // all its heads come first; CTAs start in block order as SMs free up, which
+  // makes this longest-first list scheduling within an L2-sized set of heads.
+  int bh, kv_tile;
+  if (CAUSAL) {
+    const int big = args.group_big, ubig = NT * big, nbig_units = args.num_big_groups * ubig;
+    const int u = (int)blockIdx.x;
+    int r, hg, h0;
+    if (u < nbig_units) {
+      const int g = u / ubig;
+      r = u - g * ubig;
+      hg = big;
+      h0 = g * big;
+    } else {
+      const int gs = NT * (big - 1), u2 = u - nbig_units, g = u2 / gs;
+      r = u2 - g * gs;
+      hg = big - 1;
+      h0 = args.num_big_groups * big + g * (big - 1);
+    }
+    bh = h0 + r % hg;
+    kv_tile = r / hg;
+  } else {
+    bh = (int)(blockIdx.x / (unsigned)NT);
+    kv_tile = (int)(blockIdx.x % (unsigned)NT);
+  }
   const int head_row0 = bh * args.N;
   const int kv_row0 = head_row0 + kv_tile * 128;
   const int i_begin = CAUSAL ? kv_tile : 0;  // first query tile that sees this key tile
@@ -257,11 +282,17 @@ __global__ void __launch_bounds__(384, 1)
         // A repeats the first (LBO = 0) and its output lanes are ignored.
         constexpr uint32_t kt_lbo = (D == 128) ? C::BLK : 0;
         const uint32_t tA = tmem + C::TM_A, tB = tmem + C::TM_B;
+        // Descriptors: the start address is a descriptor's low 14 bits (address /
+        // 16, below 2^14 for any shared-memory address), so each K step adds a
+        // constant to one base descriptor per operand.  The base addresses pass
+        // through an opaque move, so that the descriptors of every tile and step
+        // are not hoisted out of the loop into this thread's 56 registers.
         auto issue_kxq = [&](uint32_t dst, uint32_t a_tile, uint32_t b_tile) {  // dst = A_tile B_tile^T, K = D
+          const uint64_t da = sdesc_sw128(opaque_u32(a_tile), 16), db = sdesc_sw128(opaque_u32(b_tile), 16);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BLK + (kk & 3) * 32;
-            mma_ss(dst, sdesc_sw128(a_tile + off, 16), sdesc_sw128(b_tile + off, 16), id_s, kk > 0 ? 1u : 0u);
+            const uint32_t off16 = ((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4;
+            mma_ss(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
           }
         };
         bool ok = mbar_wait(bar_kv_full, 0, abort_flag, kSiteBwdMmaKV);
@@ -278,23 +309,29 @@ __global__ void __launch_bounds__(384, 1)
           // dV += P^T dO  (A = P^T from TMEM columns 0..63; 8 steps of 16 queries)
           if (!(ok = mbar_wait(bar_p_full, it & 1, abort_flag, kSiteBwdMmaP))) break;
           tc_fence_after();
+          {
+            const uint64_t db = sdesc_sw128(opaque_u32(sDO(s)), C::BLK);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::TM_DV, tA + kk * 8, sdesc_sw128(sDO(s) + kk * 2048, C::BLK), id_kv,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + C::TM_DV, tA + kk * 8, db + kk * (2048 >> 4), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          }
           // dK += dS^T Q  (A = dS^T from TMEM columns 64..127)
           if (!(ok = mbar_wait(bar_ds_full, it & 1, abort_flag, kSiteBwdMmaDS))) break;
           tc_fence_after();
+          {
+            const uint64_t db = sdesc_sw128(opaque_u32(sQ(s)), C::BLK);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::TM_DK, tA + 64 + kk * 8, sdesc_sw128(sQ(s) + kk * 2048, C::BLK), id_kv,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + C::TM_DK, tA + 64 + kk * 8, db + kk * (2048 >> 4), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          }
           // (the Q/dO stage is released by the dQ drain, which reuses it as staging)
           // dQ^T = K^T dS^T into region B (dP^T already read)
+          {
+            const uint64_t da = sdesc_sw128(opaque_u32(sK), kt_lbo), db = sdesc_sw128(opaque_u32(sDS), C::BLK);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tB, sdesc_sw128(sK + kk * 2048, kt_lbo), sdesc_sw128(sDS + kk * 2048, C::BLK), id_q,
-                   kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tB, da + kk * (2048 >> 4), db + kk * (2048 >> 4), id_q, kk > 0 ? 1u : 0u);
+          }
           mma_commit(bar_dq_full);
           if (it + 1 < n_it) {
             const int s1 = (it + 1) % C::NS;

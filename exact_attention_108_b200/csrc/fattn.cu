@@ -134,18 +134,17 @@ int sm_count(int* out) {
   return FATTN_OK;
 }
 
-// Causal forward: the heads' scheduling groups.  The units of a group run
-// longest first, so a group must hold enough work that its longest unit (N/128
-// key tiles) is no more than about 2/3 of what each SM gets from the group; its
-// keys and values (4*N*d bytes per head) should stay well inside L2.  The heads
-// are then split into groups whose sizes differ by at most one (a small last
-// group would leave its long units running alone at the end).
-void causal_groups(int BH, int N, int d, int sms, int* big, int* num_big) {
-  const long long nt = N / 128, np = (nt + 1) / 2;
-  long long work = 0;  // key tiles summed over the pairs of one head
-  for (long long p = 0; p < np; ++p) work += (2 * p + 2 < nt ? 2 * p + 2 : nt);
-  long long g = (3ll * sms * nt + 2 * work - 1) / (2 * work);
-  const long long cap = (48ll << 20) / (4ll * N * d);
+// Causal kernels: the heads' scheduling groups.  The units of a group run
+// longest first, so a group must hold enough work that its longest unit
+// (`longest` tile steps, out of `work` per head) is no more than about 2/3 of
+// what each SM gets from the group, while the group's per-head working set
+// (`head_bytes`) stays well inside L2.  The heads are then split into groups whose
+// sizes differ by at most one (a small last group would leave its long units
+// running alone at the end).
+void causal_groups(int BH, long long work, long long longest, long long head_bytes, int sms, int* big,
+                   int* num_big) {
+  long long g = (3ll * sms * longest + 2 * work - 1) / (2 * work);
+  const long long cap = (48ll << 20) / head_bytes;
   if (g > cap) g = cap;
   if (g > BH) g = BH;
   if (g < 1) g = 1;
@@ -217,8 +216,14 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   const int ctas = a.num_units < sms ? a.num_units : sms;  // persistent: at most one CTA per SM
   fattn::FwdArgs args = a;
   args.sched = nullptr;
-  if (CAUSAL) causal_groups(a.num_units / ((a.num_q_tiles + 1) / 2), a.N, D, sms, &args.group_big,
-                            &args.num_big_groups);
+  if (CAUSAL) {
+    // forward units: pairs of query tiles; pair p needs min(2p + 2, NT) key tiles,
+    // and a head's keys and values take 4*N*d bytes
+    const long long nt = a.num_q_tiles, np = (nt + 1) / 2;
+    long long work = 0;
+    for (long long p = 0; p < np; ++p) work += (2 * p + 2 < nt ? 2 * p + 2 : nt);
+    causal_groups(a.num_units / (int)np, work, nt, 4ll * a.N * D, sms, &args.group_big, &args.num_big_groups);
+  }
   SchedPool& pool = g_sched_pool[dev];
   std::unique_lock<std::mutex> lock(pool.mu, std::defer_lock);
   int slot = -1;
@@ -248,7 +253,18 @@ int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   constexpr int smem = fattn::BwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
   dim3 grid((unsigned)((long long)BH * a.num_tiles));
-  kern<<<grid, 384, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, a);
+  fattn::BwdArgs args = a;
+  args.group_big = 1;
+  args.num_big_groups = BH;
+  if (CAUSAL) {
+    // units: key tiles; tile t meets NT - t query tiles.  Per head the group
+    // keeps the fp32 dQ accumulator, Q and dO in L2: 8*N*d bytes.
+    int sms = 0;
+    if (int rc = sm_count(&sms)) return rc;
+    const long long nt = a.num_tiles;
+    causal_groups(BH, nt * (nt + 1) / 2, nt, 8ll * a.N * D, sms, &args.group_big, &args.num_big_groups);
+  }
+  kern<<<grid, 384, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dkdv_kernel launch");
   return FATTN_OK;
