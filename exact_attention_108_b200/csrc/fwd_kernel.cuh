@@ -339,10 +339,10 @@ __global__ void __launch_bounds__(384, 1)
               if (!(ok = mbar_wait(bar_p_full(k), tk[k] & 1, abort_flag, kSiteFwdMmaP))) break;
               tc_fence_after();
               const uint32_t tP = tmem + C::TM_S + k * 128;
+              const uint64_t dv = sdesc_sw128(opaque_u32(vaddr), C::BLK);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step = 8 TMEM columns of packed P
-                mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, sdesc_sw128(vaddr + kk * 2048, C::BLK), idPV,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+                mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, dv + kk * (2048 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
               mma_commit(bar_pv_done(k));
               ++tk[k];
               if (j + 1 < n_kv_of(k)) {
