@@ -394,40 +394,50 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(bar_s_full(k), tk & 1, abort_flag, kSiteFwdSoftS);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
+        // S_k row r -> registers in two halves of 64 keys: the row max of the first
+        // half runs while the second is still on its way from TMEM.  On the diagonal
+        // tile the keys c > r become -inf (+inf for a negative scale) first.  Row max
+        // of the raw scores, turned into the max of scale * score (log2 units); four
+        // independent three-input chains keep the dependencies short.
         uint32_t v[4][32];
-  #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tS + c4 * 32, v[c4]);
-  #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld_wait(v[c4]);
-        if (CAUSAL && j == q_tile) {
-  #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > r) v[c >> 5][c & 31] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
-        }
-        // row max of the raw scores, turned into the max of scale * score (log2 units);
-        // four independent three-input chains keep the dependencies short
+        const bool diag_tile = CAUSAL && j == q_tile;
+        const float masked = sl2 >= 0.f ? -INFINITY : INFINITY;
         float mx;
         {
-          float pm[4];
+          tmem_ld32(tS, v[0]);
+          tmem_ld32(tS + 32, v[1]);
+          tmem_ld_wait(v[0]);
+          tmem_ld_wait(v[1]);
+          tmem_ld32(tS + 64, v[2]);
+          tmem_ld32(tS + 96, v[3]);
+          float pm[4] = {masked, masked, masked, masked};
+          auto half = [&](int h) {
+            if (diag_tile) {
   #pragma unroll
-          for (int u = 0; u < 4; ++u) pm[u] = __uint_as_float(v[u][0]);
-          if (sl2 >= 0.f) {
+              for (int c = h * 64; c < h * 64 + 64; ++c)
+                if (c > r) v[c >> 5][c & 31] = __float_as_uint(masked);
+            }
+            if (sl2 >= 0.f) {
   #pragma unroll
-            for (int c = 0; c < 128; c += 8)
+              for (int c = h * 64; c < h * 64 + 64; c += 8)
   #pragma unroll
-              for (int u = 0; u < 4; ++u)
-                pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
-                              __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
-            mx = fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3]));
-          } else {
+                for (int u = 0; u < 4; ++u)
+                  pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                                __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+            } else {
   #pragma unroll
-            for (int c = 0; c < 128; c += 8)
+              for (int c = h * 64; c < h * 64 + 64; c += 8)
   #pragma unroll
-              for (int u = 0; u < 4; ++u)
-                pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
-                              __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
-            mx = fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
-          }
+                for (int u = 0; u < 4; ++u)
+                  pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                                __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+            }
+          };
+          half(0);
+          tmem_ld_wait(v[2]);
+          tmem_ld_wait(v[3]);
+          half(1);
+          mx = sl2 >= 0.f ? fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3])) : fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
           mx *= sl2;
         }
         // lazily move the reference max; rescale O and l only when it moves
