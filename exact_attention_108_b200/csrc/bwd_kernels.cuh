@@ -113,7 +113,8 @@ struct BwdCfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;  // the dynamic shared window starts 1024-byte aligned
   static constexpr int TMEM_COLS = 512;
-  // Region A: S^T, then P^T (bf16 pairs, columns 0..63) and dS^T (64..127).
+  // Region A: S^T (fp32, column = query), then per 64-query half h: P^T (bf16
+  // pairs) at columns 64h..64h+31 and dS^T at 64h+32..64h+63.
   // Region B: dP^T, then dQ^T.  Then the dV and dK accumulators.
   static constexpr int TM_A = 0, TM_B = 128, TM_DV = 256, TM_DK = 256 + D;
 };
@@ -133,14 +134,20 @@ enum : int {
 };
 
 // Roles (384 threads = three warpgroups):
-//   warps 0..3   softmax-gradient group, thread = key row of the tile: P^T, dS^T
-//   warps 4..7   dQ drain (thread = head-dim lane of dQ^T) and the dK/dV epilogue
+//   warps 0..7   gradient warps.  Warpgroup h (warps 4h..4h+3) takes queries
+//                64h..64h+63 of every query tile; thread = key row of the tile for
+//                P^T and dS^T, thread = head-dim lane for its half of dQ^T.  Warps
+//                4..7 also write dK and dV at the end.
 //   warp 8       TMA producer (K, V once; Q/dO tiles through an NS-deep ring)
-//   warp 9       tcgen05 issuer (one thread); warps 10, 11 idle
+//   warp 9       tcgen05 issuer (one thread)
+//   warp 10      dQ reducer (one thread): one bulk reduce-add per query tile
+//   warp 11      idle
 // Per query tile i the tensor cores run
 //   ... dV_i | dK_i dQ_i S_{i+1} | dP_{i+1} | dV_{i+1} | ...
 // so that the exponentials of P_{i+1} (which need only S_{i+1}) overlap the dQ
-// drain and dP_{i+1}, and dV_{i+1} overlaps the dS arithmetic.
+// drain and dP_{i+1}, and dV_{i+1} overlaps the dS arithmetic.  Splitting each
+// row's queries over two warpgroups halves the exponential and dS work on that
+// chain.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fattn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -215,13 +222,13 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_p_full, 128);
-    mbar_init(bar_ds_full, 128);
+    mbar_init(bar_p_full, 256);
+    mbar_init(bar_ds_full, 256);
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 128);
+    mbar_init(bar_dq_free, 256);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
-    mbar_init(bar_staged, 128);
+    mbar_init(bar_staged, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -306,23 +313,25 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int it = 0; it < n_it && ok; ++it) {
           const int s = it % C::NS;
-          // dV += P^T dO  (A = P^T from TMEM columns 0..63; 8 steps of 16 queries)
+          // dV += P^T dO  (A = P^T from TMEM, two 64-query halves; 8 steps of 16 queries)
           if (!(ok = mbar_wait(bar_p_full, it & 1, abort_flag, kSiteBwdMmaP))) break;
           tc_fence_after();
           {
             const uint64_t db = sdesc_sw128(opaque_u32(sDO(s)), C::BLK);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + C::TM_DV, tA + kk * 8, db + kk * (2048 >> 4), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)  // queries 16kk..: P^T of half kk/4 at columns 64*(kk/4) + 8*(kk%4)
+              mma_ts(tmem + C::TM_DV, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (2048 >> 4), id_kv,
+                     (it > 0 || kk > 0) ? 1u : 0u);
           }
-          // dK += dS^T Q  (A = dS^T from TMEM columns 64..127)
+          // dK += dS^T Q  (A = dS^T from TMEM, two 64-query halves)
           if (!(ok = mbar_wait(bar_ds_full, it & 1, abort_flag, kSiteBwdMmaDS))) break;
           tc_fence_after();
           {
             const uint64_t db = sdesc_sw128(opaque_u32(sQ(s)), C::BLK);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + C::TM_DK, tA + 64 + kk * 8, db + kk * (2048 >> 4), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)  // dS^T of half kk/4 at columns 64*(kk/4) + 32 + 8*(kk%4)
+              mma_ts(tmem + C::TM_DK, tA + (kk >> 2) * 64 + 32 + (kk & 3) * 8, db + kk * (2048 >> 4), id_kv,
+                     (it > 0 || kk > 0) ? 1u : 0u);
           }
           // (the Q/dO stage is released by the dQ drain, which reuses it as staging)
           // dQ^T = K^T dS^T into region B (dP^T already read)
@@ -353,168 +362,167 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait_ns(bar_drain, 0, 100000000ull);
       }
       __syncwarp();
+    } else if (warp == 10) {
+      // ---------------------------------------------------------- dQ reducer
+      // The gradient warps stage dQ^T_i as row-major fp32 [128 queries][D] in step
+      // i's Q/dO stage; one TMA bulk reduce-add puts it into the accumulator rows,
+      // which are contiguous.  The stage goes back to the producer once the reduce
+      // has read it, without holding up a gradient warp meanwhile.
+      if (lane == 0) {
+        for (int it = 0; it < n_it; ++it) {
+          const int s = it % C::NS;
+          if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
+          float* dst = args.dq_acc + (size_t)(head_row0 + (i_begin + it) * 128) * D;
+          bulk_reduce_add_f32(dst, sQ(s), 128 * D * 4);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(bar_q_empty(s));  // the producer may refill the stage
+        }
+        bulk_wait0();  // the last reduce has landed in global memory
+      }
+      __syncwarp();
     }
-  } else if (warp < 4) {
+  } else {
     regs_increase<224>();
-    // ------------------------------------------------- softmax-gradient group
-    const int r = warp * 32 + lane;  // key row inside the tile
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ---------------------------------------------------------- gradient warps
+    const int h = warp >> 2;   // query half: queries 64h .. 64h+63 of each tile
+    const int wq = warp & 3;   // TMEM lane quarter of this warp
+    const int r = wq * 32 + lane;  // key row (P^T, dS^T), head-dim lane (dQ^T)
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tA = tmem + C::TM_A + lane_off, tB = tmem + C::TM_B + lane_off;
     const float sl2 = args.scale_log2;
+    const bool has_d = r < D;  // TMEM lane = head-dim index of dQ^T
+    bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int s = it % C::NS;
-      bool ok = mbar_wait(bar_s_full, it & 1, abort_flag, kSiteBwdSoftS);
+      ok = mbar_wait(bar_s_full, it & 1, abort_flag, kSiteBwdSoftS);
       ok = ok && mbar_wait(bar_q_full(s), (it / C::NS) & 1, abort_flag, kSiteBwdSoftS);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      const float* lse_s = stat(s);
-      const float* dvec_s = stat(s) + 128;
+      const float* lse_s = stat(s) + 64 * h;
+      const float* dvec_s = stat(s) + 128 + 64 * h;
       const bool diag = CAUSAL && it == 0;  // queries c < r of the diagonal tile are masked
-      // P^T row: 128 queries, kept in fp32 for dS and packed to bf16 for dV
-      float p[128];
+      // P^T row, this warpgroup's 64 queries: kept in fp32 for dS, packed to bf16 for dV
+      float p[64];
       {
-        uint32_t v[4][32];
+        uint32_t v[2][32];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tA + c4 * 32, v[c4]);
+        for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(tA + 64 * h + c2 * 32, v[c2]);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld_wait(v[c4]);
+        for (int c2 = 0; c2 < 2; ++c2) tmem_ld_wait(v[c2]);
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c);  // one broadcast load per 4 columns
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float e = ex2(fmaf(__uint_as_float(v[(c + u) >> 5][(c + u) & 31]), sl2, -lv[u]));
-            p[c + u] = (diag && c + u < r) ? 0.f : e;
+            p[c + u] = (diag && 64 * h + c + u < r) ? 0.f : e;
           }
         }
       }
       {
-        uint32_t pk[2][32];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p[c], p[c + 1]);
-        tmem_st32(tA, pk[0]);
-        tmem_st32(tA + 32, pk[1]);
+        for (int c = 0; c < 64; c += 2) pk[c >> 1] = pack_bf16x2(p[c], p[c + 1]);
+        // bf16 pairs into columns 64h .. 64h+31: inside this warpgroup's own S^T
+        // columns, which the other warpgroup never reads
+        tmem_st32(tA + 64 * h, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p_full);
       // dS^T = P^T o (dP^T - D), 32 queries at a time
       ok = mbar_wait(bar_dp_full, it & 1, abort_flag, kSiteBwdSoftDP);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t dv[32];
-        tmem_ld32(tB + c4 * 32, dv);
+        tmem_ld32(tB + 64 * h + c2 * 32, dv);
         tmem_ld_wait(dv);
         uint32_t dsk[16];
 #pragma unroll
         for (int t = 0; t < 16; t += 2) {
-          const int c = c4 * 32 + 2 * t;
+          const int c = c2 * 32 + 2 * t;
           const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c);  // one broadcast load per 4 columns
           dsk[t] = pack_bf16x2(p[c] * (__uint_as_float(dv[2 * t]) - d4.x),
                                p[c + 1] * (__uint_as_float(dv[2 * t + 1]) - d4.y));
           dsk[t + 1] = pack_bf16x2(p[c + 2] * (__uint_as_float(dv[2 * t + 2]) - d4.z),
                                    p[c + 3] * (__uint_as_float(dv[2 * t + 3]) - d4.w));
         }
-        tmem_st16(tA + 64 + c4 * 16, dsk);
+        tmem_st16(tA + 64 * h + 32 + c2 * 16, dsk);  // columns 64h+32 .. 64h+63
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int ch = (c4 & 1) * 4 + q4;  // 16-byte chunk inside the 64-query block c4 / 2
-          st_shared_v4(sDS + (c4 >> 1) * C::BLK + sw128_offset(r, ch), dsk[q4 * 4], dsk[q4 * 4 + 1],
+        for (int q4 = 0; q4 < 4; ++q4)  // 16-byte chunk c2*4+q4 of the 64-query block h
+          st_shared_v4(sDS + h * C::BLK + sw128_offset(r, c2 * 4 + q4), dsk[q4 * 4], dsk[q4 * 4 + 1],
                        dsk[q4 * 4 + 2], dsk[q4 * 4 + 3]);
-        }
       }
       tmem_st_wait();
       fence_async_shared();
       tc_fence_before();
       mbar_arrive(bar_ds_full);
-    }
-    tc_fence_before();
-  } else {
-    regs_increase<224>();
-    // --------------------------------------------- dQ drain, dK/dV epilogue
-    const int wq = warp - 4;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const bool has_d = wq * 32 < D;  // TMEM lane = head-dim index of dQ^T
-    const int dcol = wq * 32 + lane;
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+      // dQ^T_i, this warpgroup's 64 queries -> shared memory as row-major fp32
+      // [128 queries][D] in this step's Q/dO stage (free: its last readers, dV_i and
+      // dK_i, completed before dQ^T_i) for the reducer's bulk reduce-add
       ok = mbar_wait(bar_dq_full, it & 1, abort_flag, kSiteBwdDrain);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      uint32_t v[4][32];
+      uint32_t v[2][32];
       if (has_d) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tmem + C::TM_B + lane_off + c4 * 32, v[c4]);
+        for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(tB + 64 * h + c2 * 32, v[c2]);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld_wait(v[c4]);
+        for (int c2 = 0; c2 < 2; ++c2) tmem_ld_wait(v[c2]);
       }
       tc_fence_before();
       mbar_arrive(bar_dq_free);
-      // dQ^T_i -> shared memory as row-major fp32 [128 queries][D] in this step's Q/dO
-      // stage (free: its last readers, dV_i and dK_i, completed before dQ^T_i) ->
-      // one TMA bulk reduce-add into the accumulator rows, which are contiguous.
-      const int s = it % C::NS;
       if (has_d) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          st_shared_f32(sQ(s) + (uint32_t)(c * D + dcol) * 4u, __uint_as_float(v[c >> 5][c & 31]));
+        for (int c = 0; c < 64; ++c)
+          st_shared_f32(sQ(s) + (uint32_t)((64 * h + c) * D + r) * 4u, __uint_as_float(v[c >> 5][c & 31]));
       }
       fence_async_shared();
       mbar_arrive(bar_staged);
-      if (wq == 0 && lane == 0) {
-        ok = mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain);
-        if (ok) {
-          float* dst = args.dq_acc + (size_t)(head_row0 + (i_begin + it) * 128) * D;
-          bulk_reduce_add_f32(dst, sQ(s), 128 * D * 4);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        mbar_arrive(bar_q_empty(s));  // the producer may refill the stage
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
     }
-    if (wq == 0 && lane == 0) bulk_wait0();  // the last reduce has landed in global memory
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, kSiteBwdEpi));
-    if (ok) {
-      tc_fence_after();
-      // dV, dK rows (thread = key row) -> bf16 -> the now idle V and K tiles -> TMA store
-      const int row = wq * 32 + lane;
+    if (h == 1) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, kSiteBwdEpi));
+      if (ok) {
+        tc_fence_after();
+        // dV, dK rows (thread = key row) -> bf16 -> the now idle V and K tiles -> TMA store
+        const int row = r;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
-        const uint32_t sdst = which ? sK : sV;
-        const float mul = which ? args.scale : 1.f;
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t tsrc = tmem + (which ? C::TM_DK : C::TM_DV) + lane_off;
+          const uint32_t sdst = which ? sK : sV;
+          const float mul = which ? args.scale : 1.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tsrc + c * 32, v);
-          tmem_ld_wait(v);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t w32[32];
+            tmem_ld32(tsrc + c * 32, w32);
+            tmem_ld_wait(w32);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = (c & 1) * 4 + q4;
-            const uint32_t* w = &v[q4 * 8];
-            st_shared_v4(sdst + (c >> 1) * C::BLK + sw128_offset(row, chunk),
-                         pack_bf16x2(__uint_as_float(w[0]) * mul, __uint_as_float(w[1]) * mul),
-                         pack_bf16x2(__uint_as_float(w[2]) * mul, __uint_as_float(w[3]) * mul),
-                         pack_bf16x2(__uint_as_float(w[4]) * mul, __uint_as_float(w[5]) * mul),
-                         pack_bf16x2(__uint_as_float(w[6]) * mul, __uint_as_float(w[7]) * mul));
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int chunk = (c & 1) * 4 + q4;
+              const uint32_t* w = &w32[q4 * 8];
+              st_shared_v4(sdst + (c >> 1) * C::BLK + sw128_offset(row, chunk),
+                           pack_bf16x2(__uint_as_float(w[0]) * mul, __uint_as_float(w[1]) * mul),
+                           pack_bf16x2(__uint_as_float(w[2]) * mul, __uint_as_float(w[3]) * mul),
+                           pack_bf16x2(__uint_as_float(w[4]) * mul, __uint_as_float(w[5]) * mul),
+                           pack_bf16x2(__uint_as_float(w[6]) * mul, __uint_as_float(w[7]) * mul));
+            }
           }
         }
-      }
-      fence_async_shared();
-      named_barrier(1, 128);
-      if (wq == 0 && lane == 0) {
+        fence_async_shared();
+        named_barrier(1, 128);
+        if (wq == 0 && lane == 0) {
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb) {
-          tma_store_2d(&tm_dv, sV + kb * C::BLK, kb * 64, kv_row0);
-          tma_store_2d(&tm_dk, sK + kb * C::BLK, kb * 64, kv_row0);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tma_store_2d(&tm_dv, sV + kb * C::BLK, kb * 64, kv_row0);
+            tma_store_2d(&tm_dk, sK + kb * C::BLK, kb * 64, kv_row0);
+          }
+          bulk_commit();
+          bulk_wait0();
         }
-        bulk_commit();
-        bulk_wait0();
       }
     }
     tc_fence_before();
