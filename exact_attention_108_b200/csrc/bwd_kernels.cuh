@@ -22,6 +22,8 @@
 //  3. fattn_bwd_dq_kernel    dQ = bf16(scale * accumulator).
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fattn {
@@ -32,13 +34,21 @@ __global__ void __launch_bounds__(256) fattn_bwd_pre_kernel(const __nv_bfloat16*
                                                             const __nv_bfloat16* __restrict__ dout,
                                                             const float* __restrict__ lse, float* __restrict__ dvec,
                                                             float* __restrict__ lse2, float* __restrict__ dq_acc,
-                                                            long long rows) {
+                                                            long long heads, int N, int NP) {
+  // One thread group per row of the padded statistics [heads][NP]: rows n < N get
+  // D = sum(dO o O) and LSE * log2(e) and have their dQ accumulator row zeroed;
+  // the padding rows of a ragged last tile get 0 (finite, and masked where used).
   constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
   constexpr int RPB = 256 / TPR;
-  const long long row = (long long)blockIdx.x * RPB + threadIdx.x / TPR;
+  const long long prow = (long long)blockIdx.x * RPB + threadIdx.x / TPR;
+  const bool in_range = prow < heads * NP;
+  const long long bh = prow / NP;
+  const int n = (int)(prow - bh * NP);
+  const bool valid = in_range && n < N;
+  const long long row = bh * N + n;
   const int part = threadIdx.x % TPR;
   float acc = 0.f;
-  if (row < rows) {
+  if (valid) {
     const size_t off = (size_t)row * D + part * 8;
     const uint4 a = *reinterpret_cast<const uint4*>(o + off);
     const uint4 b = *reinterpret_cast<const uint4*>(dout + off);
@@ -57,9 +67,9 @@ __global__ void __launch_bounds__(256) fattn_bwd_pre_kernel(const __nv_bfloat16*
   }
 #pragma unroll
   for (int w = TPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-  if (row < rows && part == 0) {
-    dvec[row] = acc;
-    lse2[row] = lse[row] * 1.4426950408889634f;
+  if (in_range && part == 0) {
+    dvec[prow] = valid ? acc : 0.f;
+    lse2[prow] = valid ? lse[row] * 1.4426950408889634f : 0.f;
   }
 }
 
@@ -83,11 +93,13 @@ __global__ void __launch_bounds__(256) fattn_bwd_dq_kernel(const float* __restri
 
 // ------------------------------------------------------------------ kernel 2
 struct BwdArgs {
-  const float* lse2;  // [B*H*N]  LSE * log2(e)
-  const float* dvec;  // [B*H*N]  D
+  const float* lse2;  // [B*H][stat_stride]  LSE * log2(e)
+  const float* dvec;  // [B*H][stat_stride]  D
   float* dq_acc;      // [B*H*N, D] fp32
   int N;
-  int num_tiles;      // N / 128
+  int num_tiles;      // ceil(N / 128)
+  int stat_stride;    // num_tiles * 128: one head's padded statistics
+  int n_tail;         // rows of the last 128-row tile, 1..128
   int group_big;      // causal order: heads in each of the first num_big_groups groups;
   int num_big_groups; //   the remaining groups hold group_big - 1 heads
   float scale;        // for dK
@@ -217,7 +229,6 @@ __global__ void __launch_bounds__(384, 1)
     kv_tile = (int)(blockIdx.x % (unsigned)NT);
   }
   const int head_row0 = bh * args.N;
-  const int kv_row0 = head_row0 + kv_tile * 128;
   const int i_begin = CAUSAL ? kv_tile : 0;  // first query tile that sees this key tile
   const int n_it = NT - i_begin;
 
@@ -262,22 +273,23 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_2d(sK + kb * C::BLK, &tm_k, bar_kv_full, kb * 64, kv_row0);
-          tma_load_2d(sV + kb * C::BLK, &tm_v, bar_kv_full, kb * 64, kv_row0);
+          tma_load_3d(sK + kb * C::BLK, &tm_k, bar_kv_full, kb * 64, kv_tile * 128, bh);
+          tma_load_3d(sV + kb * C::BLK, &tm_v, bar_kv_full, kb * 64, kv_tile * 128, bh);
         }
         int it = 0;
         for (; it < n_it; ++it) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_q_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
-          const int q_row = head_row0 + (i_begin + it) * 128;
+          const int q_tile = i_begin + it;
+          const size_t stat_row = (size_t)bh * args.stat_stride + q_tile * 128;
           mbar_arrive_expect_tx(bar_q_full(s), 2 * C::TILE + 1024);
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb) {
-            tma_load_2d(sQ(s) + kb * C::BLK, &tm_q, bar_q_full(s), kb * 64, q_row);
-            tma_load_2d(sDO(s) + kb * C::BLK, &tm_do, bar_q_full(s), kb * 64, q_row);
+            tma_load_3d(sQ(s) + kb * C::BLK, &tm_q, bar_q_full(s), kb * 64, q_tile * 128, bh);
+            tma_load_3d(sDO(s) + kb * C::BLK, &tm_do, bar_q_full(s), kb * 64, q_tile * 128, bh);
           }
-          bulk_load(sStat(s), args.lse2 + q_row, 512, bar_q_full(s));
-          bulk_load(sStat(s) + 512, args.dvec + q_row, 512, bar_q_full(s));
+          bulk_load(sStat(s), args.lse2 + stat_row, 512, bar_q_full(s));
+          bulk_load(sStat(s) + 512, args.dvec + stat_row, 512, bar_q_full(s));
         }
         if (it < n_it) {  // aborted: let the copies already issued land
           mbar_wait_ns(bar_kv_full, 0, 100000000ull);
@@ -379,8 +391,11 @@ __global__ void __launch_bounds__(384, 1)
         for (int it = 0; it < n_it; ++it) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
-          float* dst = args.dq_acc + (size_t)(head_row0 + (i_begin + it) * 128) * D;
-          bulk_reduce_add_f32(dst, sQ(s), 128 * D * 4);
+          // only the tile's rows inside the sequence (a ragged last tile has fewer)
+          const int q_tile = i_begin + it;
+          const int rows = q_tile == NT - 1 ? args.n_tail : 128;
+          float* dst = args.dq_acc + (size_t)(head_row0 + q_tile * 128) * D;
+          bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows * D * 4));
           bulk_commit();
           bulk_wait_read0();
           mbar_arrive(bar_q_empty(s));  // the producer may refill the stage
@@ -409,6 +424,14 @@ __global__ void __launch_bounds__(384, 1)
       const float* lse_s = stat(s) + 64 * h;
       const float* dvec_s = stat(s) + 128 + 64 * h;
       const bool diag = CAUSAL && it == 0;  // queries c < r of the diagonal tile are masked
+      // P = 0 outside the window lo <= c < hi of this half's 64 queries: on the
+      // diagonal tile the queries before this thread's key, in a ragged last query
+      // tile the queries past the sequence, and everything for a key past it
+      const int q_valid = i_begin + it == NT - 1 ? args.n_tail - 64 * h : 64;
+      const bool k_out = kv_tile == NT - 1 && r >= args.n_tail;
+      const int lo = diag ? r - 64 * h : 0;
+      const int hi = k_out ? 0 : q_valid;
+      const bool any_mask = __any_sync(0xffffffffu, lo > 0 || hi < 64);  // warp-uniform
       // P^T row, this warpgroup's 64 queries: kept in fp32 for dS, packed to bf16 for dV
       float p[64];
       {
@@ -417,25 +440,36 @@ __global__ void __launch_bounds__(384, 1)
         for (int c2 = 0; c2 < 2; ++c2) tmem_ld32(tA + 64 * h + c2 * 32, v[c2]);
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) tmem_ld_wait(v[c2]);
+        auto p_loop = [&](auto masked) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c);  // one broadcast load per 4 columns
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-          float e[4];
+          for (int c = 0; c < 64; c += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c);  // one broadcast load per 4 columns
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            float e[4];
 #pragma unroll
-          for (int u = 0; u < 4; u += 2) {
-            const float x0 = fmaf(__uint_as_float(v[(c + u) >> 5][(c + u) & 31]), sl2, -lv[u]);
-            const float x1 = fmaf(__uint_as_float(v[(c + u + 1) >> 5][(c + u + 1) & 31]), sl2, -lv[u + 1]);
-            if ((((c & 7) + u) >> 1) < kBwdPolyPairsPer8) {
-              f2_unpack(exp2_poly_x2(f2_pack(x0, x1)), e[u], e[u + 1]);  // on the FMA pipe
-            } else {
-              e[u] = ex2(x0);
-              e[u + 1] = ex2(x1);
+            for (int u = 0; u < 4; u += 2) {
+              const float x0 = fmaf(__uint_as_float(v[(c + u) >> 5][(c + u) & 31]), sl2, -lv[u]);
+              const float x1 = fmaf(__uint_as_float(v[(c + u + 1) >> 5][(c + u + 1) & 31]), sl2, -lv[u + 1]);
+              if ((((c & 7) + u) >> 1) < kBwdPolyPairsPer8) {
+                f2_unpack(exp2_poly_x2(f2_pack(x0, x1)), e[u], e[u + 1]);  // on the FMA pipe
+              } else {
+                e[u] = ex2(x0);
+                e[u + 1] = ex2(x1);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if constexpr (decltype(masked)::value)
+                p[c + u] = (c + u < lo || c + u >= hi) ? 0.f : e[u];
+              else
+                p[c + u] = e[u];
             }
           }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) p[c + u] = (diag && 64 * h + c + u < r) ? 0.f : e[u];
-        }
+        };
+        if (any_mask)
+          p_loop(std::true_type{});
+        else
+          p_loop(std::false_type{});
       }
       {
         uint32_t pk[32];
@@ -533,8 +567,9 @@ __global__ void __launch_bounds__(384, 1)
         if (wq == 0 && lane == 0) {
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb) {
-            tma_store_2d(&tm_dv, sV + kb * C::BLK, kb * 64, kv_row0);
-            tma_store_2d(&tm_dk, sK + kb * C::BLK, kb * 64, kv_row0);
+            // 3-D stores: rows of a ragged last key tile past the sequence are not written
+            tma_store_3d(&tm_dv, sV + kb * C::BLK, kb * 64, kv_tile * 128, bh);
+            tma_store_3d(&tm_dk, sK + kb * C::BLK, kb * 64, kv_tile * 128, bh);
           }
           bulk_commit();
           bulk_wait0();

@@ -57,21 +57,23 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D view [rows, cols] of a row-major bf16 or fp32 tensor, box [box_rows, box_cols],
-// 128-byte swizzle when the box row is 128 bytes wide.
-int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows,
-             uint64_t cols, uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swz) {
+// 3-D view [B*H][N][d] of a contiguous bf16 [B, H, N, d] tensor, box [1][128][64]
+// with 128-byte swizzle: one box is 64 columns of a 128-row tile of one head.
+// Rows past N inside a head read as zero and are never written, so a ragged last
+// tile needs no special copy.
+int make_head_map(CUtensorMap* map, const void* base, uint64_t heads, uint64_t N, int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     t_last_cuda_error = "cuTensorMapEncodeTiled entry point not available";
     return FATTN_ERR_CUDA;
   }
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint64_t dims[3] = {(cuuint64_t)d, N, heads};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, N * (cuuint64_t)d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[96];
     snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
@@ -81,21 +83,16 @@ int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int ele
   return FATTN_OK;
 }
 
-// bf16 [rows, d] viewed in boxes of 64 columns x box_rows rows, 128-byte swizzle.
-int make_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int d, uint32_t box_rows = 128) {
-  return make_map(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, (uint64_t)d, box_rows, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Sequence length rounded up to whole 128-row tiles.
+long long padded_n(int N) { return ((long long)N + 127) / 128 * 128; }
 
 int check_shape(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1) return FATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
-  if (N % 128 != 0) return FATTN_ERR_UNSUPPORTED;
-  const long long rows = (long long)B * H * N;
-  if (rows >= (1ll << 31)) return FATTN_ERR_UNSUPPORTED;
-  if (rows / 128 > 0x7fffffffll) return FATTN_ERR_UNSUPPORTED;  // 128-row tiles are counted in int
+  // rows, and rows rounded up to whole tiles per head, are counted in int
+  if ((long long)B * H * padded_n(N) >= (1ll << 31)) return FATTN_ERR_UNSUPPORTED;
   return FATTN_OK;
 }
 
@@ -276,22 +273,33 @@ struct WsParts {
   float* dq_acc;
 };
 
-WsParts split_workspace(void* workspace, long long rows) {
+// Workspace: D and LSE*log2(e) per query row, each head padded to whole 128-row
+// tiles ([B*H][ceil(N/128)*128] fp32, so that every tile's statistics are one
+// aligned 512-byte block), then the fp32 dQ accumulator [B*H*N, d].
+size_t ws_bytes_needed(long long heads, int N, int d) {
+  const size_t stat = align256((size_t)(heads * padded_n(N)) * sizeof(float));
+  return 2 * stat + align256((size_t)heads * N * d * sizeof(float));
+}
+
+WsParts split_workspace(void* workspace, long long heads, int N) {
   char* ws = static_cast<char*>(workspace);
+  const size_t stat = align256((size_t)(heads * padded_n(N)) * sizeof(float));
   WsParts p;
   p.dvec = reinterpret_cast<float*>(ws);
-  p.lse2 = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
-  p.dq_acc = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+  p.lse2 = reinterpret_cast<float*>(ws + stat);
+  p.dq_acc = reinterpret_cast<float*>(ws + 2 * stat);
   return p;
 }
 
 template <int D>
-int launch_pre(const void* o, const void* dout, const float* lse, long long rows, const WsParts& w, cudaStream_t st) {
+int launch_pre(const void* o, const void* dout, const float* lse, long long heads, int N, const WsParts& w,
+               cudaStream_t st) {
   constexpr int rpb = 256 / (D / 8);
-  const long long blocks = (rows + rpb - 1) / rpb;
+  const int np = (int)padded_n(N);
+  const long long blocks = (heads * np + rpb - 1) / rpb;
   fattn::fattn_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
                                                                     static_cast<const __nv_bfloat16*>(dout), lse,
-                                                                    w.dvec, w.lse2, w.dq_acc, rows);
+                                                                    w.dvec, w.lse2, w.dq_acc, heads, N, np);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_pre_kernel launch");
   return FATTN_OK;
@@ -300,20 +308,22 @@ int launch_pre(const void* o, const void* dout, const float* lse, long long rows
 template <int D>
 int launch_dkdv_d(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
                   int N, int causal, float scale, const WsParts& w, cudaStream_t st) {
-  const long long rows = (long long)B * H * N;
+  const uint64_t heads = (uint64_t)B * H;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if (int rc = make_bf16_tile_map(&mq, q, rows, D)) return rc;
-  if (int rc = make_bf16_tile_map(&mdo, dout, rows, D)) return rc;
-  if (int rc = make_bf16_tile_map(&mk, k, rows, D)) return rc;
-  if (int rc = make_bf16_tile_map(&mv, v, rows, D)) return rc;
-  if (int rc = make_bf16_tile_map(&mdk, dk, rows, D)) return rc;
-  if (int rc = make_bf16_tile_map(&mdv, dv, rows, D)) return rc;
+  if (int rc = make_head_map(&mq, q, heads, N, D)) return rc;
+  if (int rc = make_head_map(&mdo, dout, heads, N, D)) return rc;
+  if (int rc = make_head_map(&mk, k, heads, N, D)) return rc;
+  if (int rc = make_head_map(&mv, v, heads, N, D)) return rc;
+  if (int rc = make_head_map(&mdk, dk, heads, N, D)) return rc;
+  if (int rc = make_head_map(&mdv, dv, heads, N, D)) return rc;
   fattn::BwdArgs a;
   a.lse2 = w.lse2;
   a.dvec = w.dvec;
   a.dq_acc = w.dq_acc;
   a.N = N;
-  a.num_tiles = N / 128;
+  a.num_tiles = (N + 127) / 128;
+  a.stat_stride = (int)padded_n(N);
+  a.n_tail = N - (a.num_tiles - 1) * 128;
   a.scale = scale;
   a.scale_log2 = scale * kLog2e;
   const int BH = B * H;
@@ -335,9 +345,7 @@ int launch_dq(void* dq, long long rows, float scale, const WsParts& w, cudaStrea
 int check_workspace(void* workspace, size_t bytes, int B, int H, int N, int d) {
   if (!workspace) return FATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FATTN_ERR_ALIGNMENT;
-  const long long rows = (long long)B * H * N;
-  const size_t need = 2 * align256(rows * sizeof(float)) + align256(rows * (size_t)d * sizeof(float));
-  if (bytes < need) return FATTN_ERR_INVALID_ARG;
+  if (bytes < ws_bytes_needed((long long)B * H, N, d)) return FATTN_ERR_INVALID_ARG;
   return FATTN_OK;
 }
 
@@ -357,7 +365,7 @@ const char* fattn_status_string(int status) {
   switch (status) {
     case FATTN_OK: return "ok";
     case FATTN_ERR_INVALID_ARG: return "invalid argument";
-    case FATTN_ERR_UNSUPPORTED: return "unsupported shape (need d in {64,128}, N % 128 == 0)";
+    case FATTN_ERR_UNSUPPORTED: return "unsupported shape (need d in {64,128} and B*H*ceil(N/128)*128 < 2^31)";
     case FATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case FATTN_ERR_CUDA: return "CUDA error (see fattn_last_cuda_error)";
     case FATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";
@@ -390,18 +398,19 @@ int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FATTN_ERR_ALIGNMENT;
 
-  const uint64_t rows = (uint64_t)B * H * N;
+  const uint64_t heads = (uint64_t)B * H;
   CUtensorMap mq, mk, mv;
-  if (int rc = make_bf16_tile_map(&mq, q, rows, d)) return rc;
-  if (int rc = make_bf16_tile_map(&mk, k, rows, d)) return rc;
-  if (int rc = make_bf16_tile_map(&mv, v, rows, d)) return rc;
+  if (int rc = make_head_map(&mq, q, heads, N, d)) return rc;
+  if (int rc = make_head_map(&mk, k, heads, N, d)) return rc;
+  if (int rc = make_head_map(&mv, v, heads, N, d)) return rc;
 
   fattn::FwdArgs a;
   a.lse = lse;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.N = N;
-  a.num_q_tiles = N / 128;
-  a.num_units = B * H * ((N / 128 + 1) / 2);
+  a.num_q_tiles = (N + 127) / 128;
+  a.n_tail = N - (a.num_q_tiles - 1) * 128;
+  a.num_units = B * H * ((a.num_q_tiles + 1) / 2);
   a.group_big = 1;
   a.num_big_groups = 1;
   a.sched = nullptr;
@@ -426,8 +435,7 @@ int fattn_exp2_poly(const float* x, float* y, long long n, fattn_stream_t stream
 
 size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d) != FATTN_OK) return 0;
-  const size_t rows = (size_t)B * H * N;
-  return 2 * align256(rows * sizeof(float)) + align256(rows * (size_t)d * sizeof(float));
+  return ws_bytes_needed((long long)B * H, N, d);
 }
 
 int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
@@ -436,10 +444,10 @@ int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int 
   if (int rc = check_common(B, H, N, d, 1.f, 0)) return rc;
   if (!aligned16(o) || !aligned16(dout) || !aligned16(lse)) return FATTN_ERR_ALIGNMENT;
   if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
-  const long long rows = (long long)B * H * N;
-  const WsParts w = split_workspace(workspace, rows);
+  const long long heads = (long long)B * H;
+  const WsParts w = split_workspace(workspace, heads, N);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_pre<64>(o, dout, lse, rows, w, st) : launch_pre<128>(o, dout, lse, rows, w, st);
+  return d == 64 ? launch_pre<64>(o, dout, lse, heads, N, w, st) : launch_pre<128>(o, dout, lse, heads, N, w, st);
 }
 
 int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
@@ -450,7 +458,7 @@ int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
     return FATTN_ERR_ALIGNMENT;
   if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
-  const WsParts w = split_workspace(workspace, (long long)B * H * N);
+  const WsParts w = split_workspace(workspace, (long long)B * H, N);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? launch_dkdv_d<64>(q, k, v, dout, dk, dv, B, H, N, causal, scale, w, st)
                  : launch_dkdv_d<128>(q, k, v, dout, dk, dv, B, H, N, causal, scale, w, st);
@@ -463,7 +471,7 @@ int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale, void* worksp
   if (!aligned16(dq)) return FATTN_ERR_ALIGNMENT;
   if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
   const long long rows = (long long)B * H * N;
-  const WsParts w = split_workspace(workspace, rows);
+  const WsParts w = split_workspace(workspace, (long long)B * H, N);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? launch_dq<64>(dq, rows, scale, w, st) : launch_dq<128>(dq, rows, scale, w, st);
 }

@@ -40,8 +40,9 @@ namespace fattn {
 struct FwdArgs {
   float* lse;            // [B*H*N] fp32
   __nv_bfloat16* o;      // [B*H*N, D] bf16
-  int N;                 // keys per head (multiple of 128)
-  int num_q_tiles;       // N / 128
+  int N;                 // keys (and queries) per head
+  int num_q_tiles;       // ceil(N / 128)
+  int n_tail;            // rows of the last 128-row tile, 1..128
   int num_units;         // B*H * ceil(num_q_tiles / 2)
   int group_big;         // causal order: heads in each of the first num_big_groups groups;
   int num_big_groups;    //   the remaining groups hold group_big - 1 heads
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(384, 1)
   const int NP = (NT + 1) >> 1;
   const bool dyn = CAUSAL && args.sched != nullptr;
   struct Unit {
-    int head_row0, tile0, n_kv0, n_kv1, n_kv;
+    int bh, head_row0, tile0, n_kv0, n_kv1, n_kv;
   };
   auto unit_of = [&](int u) {
     Unit w;
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(384, 1)
       bh = u / NP;
       pair = u % NP;
     }
+    w.bh = bh;
     w.head_row0 = bh * args.N;
     w.tile0 = 2 * pair;
     const bool has_q1 = w.tile0 + 1 < NT;
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(384, 1)
               const uint32_t dst = sSlot0 + s * C::TILE;
 #pragma unroll
               for (int kb = 0; kb < C::KB; ++kb)
-                tma_load_2d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, w.head_row0 + j * 128);
+                tma_load_3d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, j * 128, w.bh);
               ++it;
               // Q0 after K_0, Q1 after V_0: each into the Q buffer freed longest ago
               if (j == 0 && t < nq) {
@@ -253,8 +255,7 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive_expect_tx(bar_q_full(b), C::TILE);
 #pragma unroll
                 for (int kb = 0; kb < C::KB; ++kb)
-                  tma_load_2d(sQ(b) + kb * C::BLK, &tm_q, bar_q_full(b), kb * 64,
-                              w.head_row0 + (w.tile0 + t) * 128);
+                  tma_load_3d(sQ(b) + kb * C::BLK, &tm_q, bar_q_full(b), kb * 64, (w.tile0 + t) * 128, w.bh);
                 ++qs;
               }
             }
@@ -401,6 +402,10 @@ __global__ void __launch_bounds__(384, 1)
         // independent three-input chains keep the dependencies short.
         uint32_t v[4][32];
         const bool diag_tile = CAUSAL && j == q_tile;
+        // a ragged last key tile: its keys c >= n_tail are past the sequence (their
+        // rows read as zero).  Causal rows never see them: the diagonal mask covers
+        // every key past a valid query.
+        const bool tail_tile = !CAUSAL && j == NT - 1 && args.n_tail < 128;
         const float masked = sl2 >= 0.f ? -INFINITY : INFINITY;
         float mx;
         {
@@ -416,6 +421,11 @@ __global__ void __launch_bounds__(384, 1)
   #pragma unroll
               for (int c = h * 64; c < h * 64 + 64; ++c)
                 if (c > r) v[c >> 5][c & 31] = __float_as_uint(masked);
+            }
+            if (tail_tile) {
+  #pragma unroll
+              for (int c = h * 64; c < h * 64 + 64; ++c)
+                if (c >= args.n_tail) v[c >> 5][c & 31] = __float_as_uint(masked);
             }
             if (sl2 >= 0.f) {
   #pragma unroll
@@ -508,21 +518,24 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < D / 32; ++c) tmem_ld_wait(o[c]);
       tc_fence_before();
       mbar_arrive(bar_o_free(k));  // O_k may now be overwritten by the next unit
-      // O row (bf16) straight to global memory, LSE (natural log) beside it
-      const float inv_l = 1.f / l;
-      const size_t row = (size_t)(w.head_row0 + q_tile * 128 + r);
-      uint4* dst = reinterpret_cast<uint4*>(args.o + row * D);
+      // O row (bf16) straight to global memory, LSE (natural log) beside it; rows
+      // of a ragged last tile past the sequence are not written
+      if (q_tile * 128 + r < args.N) {
+        const float inv_l = 1.f / l;
+        const size_t row = (size_t)(w.head_row0 + q_tile * 128 + r);
+        uint4* dst = reinterpret_cast<uint4*>(args.o + row * D);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c)
+        for (int c = 0; c < D / 32; ++c)
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t* x = &o[c][q4 * 8];
-          dst[c * 4 + q4] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
-        }
-      args.lse[row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t* x = &o[c][q4 * 8];
+            dst[c * 4 + q4] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
+                                         pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
+                                         pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
+                                         pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
+          }
+        args.lse[row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      }
     }
     tc_fence_before();
   }

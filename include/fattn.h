@@ -26,8 +26,11 @@
  * All pointers are DEVICE pointers on the current CUDA device and must be
  * 16-byte aligned.  Outputs must not alias inputs.
  *
- * Supported shapes: B, H, N >= 1; N % 128 == 0; d in {64, 128};
- * B * H * N < 2^31.  scale must be finite (any sign).
+ * Supported shapes: B, H, N >= 1 (any N); d in {64, 128};
+ * B * H * ceil(N / 128) * 128 < 2^31.  scale must be finite (any sign).  The
+ * kernels work on 128-row tiles; a ragged last tile of each head is masked
+ * (keys past N never receive weight, and rows past N are neither read nor
+ * written).
  *
  * Ownership and asynchrony.  The caller allocates and owns every buffer,
  * including the backward workspace.  The library allocates no device memory at
@@ -60,7 +63,7 @@ typedef struct CUstream_st* fattn_stream_t; /* same object as cudaStream_t */
 typedef enum {
   FATTN_OK = 0,
   FATTN_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, non-finite scale, too small workspace */
-  FATTN_ERR_UNSUPPORTED = 2,    /* d not in {64,128}, N % 128 != 0, size overflow */
+  FATTN_ERR_UNSUPPORTED = 2,    /* d not in {64,128}, size overflow */
   FATTN_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
   FATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed; see fattn_last_cuda_error() */
   FATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out */
@@ -87,8 +90,10 @@ int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /*
  * Bytes of device workspace fattn_bwd needs for this shape (0 for an invalid
- * shape).  Layout inside (each part 256-byte aligned): D [B,H,N] fp32,
- * LSE*log2(e) [B,H,N] fp32, fp32 dQ accumulator [B,H,N,d].
+ * shape).  Layout inside (each part 256-byte aligned): D [B*H][Np] fp32 and
+ * LSE*log2(e) [B*H][Np] fp32, where Np = ceil(N / 128) * 128 (each head padded
+ * to whole 128-row tiles, padding rows 0), then the fp32 dQ accumulator
+ * [B,H,N,d].
  */
 size_t fattn_bwd_workspace_size(int B, int H, int N, int d);
 

@@ -58,8 +58,9 @@ def test_fwd_validation(lib):
     assert _fwd(lib, N=0) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, d=96) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED
-    assert _fwd(lib, N=100) == binding.FATTN_ERR_UNSUPPORTED       # ragged length
     assert _fwd(lib, B=1 << 14, H=1 << 10, N=1 << 8) == binding.FATTN_ERR_UNSUPPORTED  # 2^32 rows
+    # 2^23 heads of 129 rows: under 2^31 rows, but 2^31 once each head is padded to whole tiles
+    assert _fwd(lib, B=1 << 13, H=1 << 10, N=129) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd(lib, scale=float("inf")) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, scale=float("nan")) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, causal=2) == binding.FATTN_ERR_INVALID_ARG
@@ -70,16 +71,17 @@ def test_fwd_validation(lib):
 def test_workspace_size(lib):
     def a256(x):
         return (x + 255) // 256 * 256
-    for (B, H, N, d) in [(1, 1, 128, 64), (4, 32, 4096, 128), (3, 5, 384, 128)]:
-        rows = B * H * N
-        assert lib.fattn_bwd_workspace_size(B, H, N, d) == 2 * a256(rows * 4) + a256(rows * d * 4)
-    assert lib.fattn_bwd_workspace_size(1, 1, 100, 64) == 0
+    # D and LSE*log2(e) per head padded to whole 128-row tiles, then the fp32 dQ accumulator
+    for (B, H, N, d) in [(1, 1, 128, 64), (4, 32, 4096, 128), (3, 5, 384, 128), (1, 1, 100, 64), (2, 3, 200, 128)]:
+        padded = B * H * ((N + 127) // 128 * 128)
+        assert lib.fattn_bwd_workspace_size(B, H, N, d) == 2 * a256(padded * 4) + a256(B * H * N * d * 4)
     assert lib.fattn_bwd_workspace_size(1, 1, 128, 96) == 0
+    assert lib.fattn_bwd_workspace_size(1, 1, 0, 64) == 0
 
 
 def _bwd(lib, ws=P, ws_bytes=None, d=64, N=128, **kw):
     if ws_bytes is None:
-        ws_bytes = lib.fattn_bwd_workspace_size(1, 1, N, d) if d in (64, 128) and N % 128 == 0 else 1 << 30
+        ws_bytes = lib.fattn_bwd_workspace_size(1, 1, N, d) if d in (64, 128) else 1 << 30
     args = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P)
     args.update(kw)
     return lib.fattn_bwd(args["q"], args["k"], args["v"], args["o"], args["do"], args["lse"], args["dq"],
@@ -91,7 +93,7 @@ def test_bwd_validation(lib):
     assert _bwd(lib, ws=None) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, ws_bytes=16) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, d=32) == binding.FATTN_ERR_UNSUPPORTED
-    assert _bwd(lib, N=200) == binding.FATTN_ERR_UNSUPPORTED
+    assert _bwd(lib, N=200, ws_bytes=lib.fattn_bwd_workspace_size(1, 1, 200, 64) - 16) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, dq=P + 2) == binding.FATTN_ERR_ALIGNMENT
     assert _bwd(lib, ws=P + 16) == binding.FATTN_ERR_ALIGNMENT  # workspace wants 256 bytes
 
