@@ -4,8 +4,9 @@
 // log-sum-exp instead of reading a stored probability matrix (page 2 "四、反向
 // 传播选择重计算而非全量保存").  Three kernels run in order on one stream:
 //
-//  1. fattn_bwd_pre_kernel   D_i = sum_c dO_ic O_ic, LSE2_i = LSE_i log2(e),
-//                            and zero the fp32 dQ accumulator.     (HBM-bound)
+//  1. fattn_bwd_pre_kernel   D_i = sum_c dO_ic O_ic, LSE2_i = LSE_i log2(e)
+//                            (per head padded to whole 128-row tiles), and
+//                            zero the fp32 dQ accumulator.         (HBM-bound)
 //  2. fattn_bwd_dkdv_kernel  one CTA per (batch*head, 128-row key tile j);
 //                            loops over the 128-row query tiles i that can see
 //                            tile j and, on the tcgen05 tensor cores,
@@ -19,6 +20,9 @@
 //                                  added into the fp32 accumulator by one TMA
 //                                  bulk reduce per query tile
 //                            (atomic global updates, page 3 "5.3 专用指令利用").
+//                            A ragged last tile (N not a multiple of 128) is
+//                            read as zeros past N through 3-D tensor maps; P
+//                            is 0 for its queries and keys past N.
 //  3. fattn_bwd_dq_kernel    dQ = bf16(scale * accumulator).
 #pragma once
 

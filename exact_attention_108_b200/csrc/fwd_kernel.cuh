@@ -25,6 +25,11 @@
 // Tensor memory (512 columns x 128 lanes): S0 at column 0, S1 at 128 (P_k, bf16,
 // overlays the first 64 columns of S_k), O0 at 256, O1 at 256 + D.
 //
+// Any N: the tiles stay 128 rows, and the 3-D tensor maps read a ragged last
+// tile's rows past N as zero.  Its keys past N are masked (non-causal; the causal
+// mask already hides them from every query before N), and its rows past N are
+// not stored.
+//
 // Online softmax with a lazily updated reference max: each row keeps a
 // reference m_ref (log2 units) and sums exp2(s - m_ref).  When a tile's row max
 // exceeds m_ref by more than kRescaleThreshold, m_ref moves up and the partial
@@ -90,7 +95,6 @@ enum : int {  // wait sites recorded in the device status word on a timeout
   kSiteFwdProducer = 0x101,
   kSiteFwdMmaQ = 0x102,
   kSiteFwdMmaK = 0x103,
-  kSiteFwdMmaPV = 0x104,
   kSiteFwdMmaP = 0x105,
   kSiteFwdMmaV = 0x106,
   kSiteFwdSoftS = 0x107,
