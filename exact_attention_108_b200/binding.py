@@ -27,7 +27,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20  # FATTN_NOALLOC_SCRATCH_BYTES
 # Every symbol include/fattn.h declares (checked by the CPU test suite).
 EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_bwd_preprocess",
             "fattn_bwd_dkdv", "fattn_bwd_dq", "fattn_status_string", "fattn_last_cuda_error",
-            "fattn_device_status", "fattn_version", "fattn_exp2_poly", "fattn_bwd_noalloc")
+            "fattn_device_status", "fattn_version", "fattn_bwd_noalloc")
 
 _lib = None
 
@@ -70,8 +70,6 @@ def load():
     L.fattn_last_cuda_error.restype = ctypes.c_char_p
     L.fattn_device_status.argtypes = [i]
     L.fattn_device_status.restype = i
-    L.fattn_exp2_poly.argtypes = [vp, vp, ctypes.c_longlong, vp]
-    L.fattn_exp2_poly.restype = i
     L.fattn_version.argtypes = []
     L.fattn_version.restype = i
     _lib = L
@@ -195,16 +193,6 @@ def bwd_dq(dq, workspace, scale: float | None = None, stream=None):
                              _nbytes(workspace), _stream_handle(stream))
     if rc != FATTN_OK:
         raise FattnError(rc, "fattn_bwd_dq")
-
-
-def exp2_poly(x, out=None, stream=None):
-    """Diagnostics: the library's FMA-pipe 2^x approximation on a CUDA fp32 tensor."""
-    _check(x, "x", torch.float32)
-    out = torch.empty_like(x) if out is None else out
-    rc = load().fattn_exp2_poly(x.data_ptr(), out.data_ptr(), x.numel(), _stream_handle(stream))
-    if rc != FATTN_OK:
-        raise FattnError(rc, "fattn_exp2_poly")
-    return out
 
 
 def bwd_noalloc(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,

@@ -149,13 +149,6 @@ enum : int {
   kSiteBwdAlign = 0x20b,
 };
 
-// Exponentials of the backward's P evaluated on the FMA pipe (exp2_poly_x2, relative
-// error 1.02e-4, far below the bf16 rounding of P and dS) per 8 columns; the rest
-// use MUFU ex2.  Both gradient warpgroups share each sub-partition's MUFU unit, but
-// on B200 moving 25% of the exponentials changes the backward by under 1% and 50%
-// makes it slower, so the share is 0.
-constexpr int kBwdPolyPairsPer8 = 0;
-
 // Roles (384 threads = three warpgroups):
 //   warps 0..7   gradient warps.  Warpgroup h (warps 4h..4h+3) takes queries
 //                64h..64h+63 of every query tile; thread = key row of the tile for
@@ -451,16 +444,8 @@ __global__ void __launch_bounds__(384, 1)
             const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
             float e[4];
 #pragma unroll
-            for (int u = 0; u < 4; u += 2) {
-              const float x0 = fmaf(__uint_as_float(v[(c + u) >> 5][(c + u) & 31]), sl2, -lv[u]);
-              const float x1 = fmaf(__uint_as_float(v[(c + u + 1) >> 5][(c + u + 1) & 31]), sl2, -lv[u + 1]);
-              if ((((c & 7) + u) >> 1) < kBwdPolyPairsPer8) {
-                f2_unpack(exp2_poly_x2(f2_pack(x0, x1)), e[u], e[u + 1]);  // on the FMA pipe
-              } else {
-                e[u] = ex2(x0);
-                e[u + 1] = ex2(x1);
-              }
-            }
+            for (int u = 0; u < 4; ++u)
+              e[u] = ex2(fmaf(__uint_as_float(v[(c + u) >> 5][(c + u) & 31]), sl2, -lv[u]));
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               if constexpr (decltype(masked)::value)

@@ -15,19 +15,6 @@
 #include "bwd_kernels.cuh"
 #include "fwd_kernel.cuh"
 
-namespace fattn {
-__global__ void fattn_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
-  for (long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x); i < n;
-       i += 2ll * gridDim.x * blockDim.x) {
-    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.f;
-    float y0, y1;
-    sm100::f2_unpack(sm100::exp2_poly_x2(sm100::f2_pack(x0, x1)), y0, y1);
-    y[i] = y0;
-    if (i + 1 < n) y[i + 1] = y1;
-  }
-}
-}  // namespace fattn
-
 namespace {
 
 thread_local std::string t_last_cuda_error;
@@ -193,10 +180,14 @@ int sched_slot(SchedPool& pool, cudaStream_t st) {
   }
   for (int i = 0; i < kSchedSlots; ++i) {
     const int s = (pool.next + i) % kSchedSlots;
-    if (cudaEventQuery(pool.ev[s]) == cudaSuccess) {
+    const cudaError_t q = cudaEventQuery(pool.ev[s]);
+    if (q == cudaSuccess) {
       pool.next = (s + 1) % kSchedSlots;
       return s;
     }
+    // a busy slot: clear the not-ready status if the runtime kept it as the last
+    // error, but leave any other pending error for the launch check to report
+    if (q == cudaErrorNotReady && cudaPeekAtLastError() == cudaErrorNotReady) (void)cudaGetLastError();
   }
   return -1;
 }
@@ -231,7 +222,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   }
   kern<<<dim3((unsigned)ctas), 384, smem, st>>>(mq, mk, mv, args);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess && e != cudaErrorNotReady) return cuda_fail(e, "fattn_fwd_kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_fwd_kernel launch");
   if (slot >= 0) {
     e = cudaEventRecord(pool.ev[slot], st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -418,19 +409,6 @@ int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, a, st) : launch_fwd<64, false>(mq, mk, mv, a, st);
   return causal ? launch_fwd<128, true>(mq, mk, mv, a, st) : launch_fwd<128, false>(mq, mk, mv, a, st);
-}
-
-int fattn_exp2_poly(const float* x, float* y, long long n, fattn_stream_t stream) {
-  if (n < 0 || ((!x || !y) && n > 0)) return FATTN_ERR_INVALID_ARG;
-  if (n == 0) return FATTN_OK;
-  if (!aligned16(x) || !aligned16(y)) return FATTN_ERR_ALIGNMENT;
-  long long blocks = (n / 2 + 255) / 256;
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  if (blocks < 1) blocks = 1;
-  fattn::fattn_exp2_poly_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "fattn_exp2_poly_kernel launch");
-  return FATTN_OK;
 }
 
 size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {

@@ -86,10 +86,6 @@ struct FwdCfg {
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: weights stay below 256
-// Exponentials evaluated on the FMA pipe (exp2_poly_x2) per 8 pairs of columns;
-// the rest use MUFU ex2.  On B200 at this tile shape the extra FMA-pipe
-// instructions cost about what they save on MUFU, so the share is 0.
-constexpr int kPolyPairsPer8 = 0;
 
 enum : int {  // wait sites recorded in the device status word on a timeout
   kSiteFwdProducer = 0x101,
@@ -473,7 +469,13 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         }
-        const bool diag = CAUSAL && j == q_tile;  // keys c > r of this tile are masked
+        // Keys c >= lim of this tile get weight 0, by a select after the exponential:
+        // the masked raw scores were set to -inf (+inf for a negative scale), and
+        // with scale 0 the product -inf * 0 is NaN, so the exponential alone cannot
+        // be trusted to give 0.  Causal: the diagonal tile, lim = r + 1; otherwise a
+        // ragged last tile, lim = n_tail.
+        const bool clip = CAUSAL ? diag_tile : tail_tile;
+        const int lim = CAUSAL ? r + 1 : args.n_tail;
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
         uint32_t pk[2][32];                          // P row as packed bf16 pairs
@@ -482,18 +484,12 @@ __global__ void __launch_bounds__(384, 1)
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
                                              __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
                                      sl2x2, negm2);
-          float p0, p1;
-          if (((c >> 1) & 7) < kPolyPairsPer8) {
-            f2_unpack(exp2_poly_x2(x2), p0, p1);  // on the FMA pipe
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          if (diag) {
-            p0 = (c > r) ? 0.f : p0;
-            p1 = (c + 1 > r) ? 0.f : p1;
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (clip) {
+            p0 = (c < lim) ? p0 : 0.f;
+            p1 = (c + 1 < lim) ? p1 : 0.f;
           }
           acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
           pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);

@@ -336,35 +336,6 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of floats on the FMA pipe (so that the MUFU unit, which the
-// softmax otherwise saturates, can be offloaded).  Method: Cody-Waite style
-// range reduction x = n + f with n = nearest integer (obtained by adding
-// 1.5 * 2^23, which leaves n in the low mantissa bits) and f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial whose coefficients are the minimax fit of
-// relative error on [-1/2, 1/2] with p(0) = 1 (fitted by linear programming in
-// csrc/fit_exp2_poly.py; max relative error 1.02e-4 in fp32); 2^n applied by
-// adding n to the exponent field.  Inputs below -64 are clamped to -64
-// (2^-64 is negligible next to the row sums, which are >= 1).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-  constexpr float kC1 = 0.6932829022407532f, kC2 = 0.24221095442771912f, kC3 = 0.055008936673402786f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -64.f), fmaxf(x1, -64.f));
-  const uint64_t t = f2_add(xc, f2_pack(kRound, kRound));
-  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
-  const uint64_t fr = f2_fma(n, f2_pack(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(fr, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
-  p = f2_fma(p, fr, f2_pack(kC1, kC1));
-  p = f2_fma(p, fr, f2_pack(1.f, 1.f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-  return f2_pack(r0, r1);
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");

@@ -37,7 +37,10 @@
  * run time.  Its only device state is static: 16 pairs of scheduling counters
  * for the causal forward, and the scratch array of fattn_bwd_noalloc.  It also
  * keeps 16 CUDA events per device, created by the first causal forward on that
- * device.  Every call only enqueues work on `stream` and returns; results are
+ * device; these and the static arrays' device addresses are looked up once per
+ * device, so the library must not be used across a reset of a device's context
+ * (cudaDeviceReset, or the primary context released and created again).  Every
+ * call only enqueues work on `stream` and returns; results are
  * valid once the stream has been synchronised.  Inputs must stay alive until
  * then.
  *
@@ -123,13 +126,18 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o,
  * workspace.  The scratch space fattn_bwd takes from its workspace comes
  * instead from one fixed array of FATTN_NOALLOC_SCRATCH_BYTES bytes (32 MiB)
  * that the library keeps in device memory; every GPU that loads the library
- * holds that array until the process exits.  Shapes whose workspace
- * (fattn_bwd_workspace_size) is larger are rejected with
- * FATTN_ERR_SCRATCH_TOO_SMALL before anything is enqueued: at d = 128 that is
- * B*H*N > 64512, at d = 64 B*H*N > 126976.
+ * holds that array until the process exits.  A shape is accepted exactly when
+ * fattn_bwd_workspace_size(B, H, N, d) <= FATTN_NOALLOC_SCRATCH_BYTES; larger
+ * ones are rejected with FATTN_ERR_SCRATCH_TOO_SMALL before anything is
+ * enqueued.  For N a multiple of 128 that means B*H*N <= 64512 at d = 128 and
+ * B*H*N <= 126976 at d = 64; for other N the per-head statistics are padded to
+ * whole 128-row tiles and count too, so the limit on B*H*N is lower.
  *
  * The first call on a device looks up the array's device address and caches
- * it; make that first call before any stream capture on that device.  All calls
+ * it; make that first call before any stream capture on that device.  The
+ * cached address belongs to the device's current context: the library must not
+ * be used across a reset of that context (cudaDeviceReset, or the primary
+ * context released and created again), which would leave it stale.  All calls
  * on one device share the array, and each call re-initialises what must start
  * at zero, so calls whose executions overlap on the GPU (on different streams,
  * or from several host threads) race on it and must be serialised by the caller.
@@ -160,17 +168,6 @@ int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout
                    void* workspace, size_t workspace_bytes, fattn_stream_t stream);
 int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale,
                  void* workspace, size_t workspace_bytes, fattn_stream_t stream);
-
-/*
- * Diagnostics: y[i] = 2^x[i] evaluated with the FMA-pipe approximation the
- * softmax loops can use for part of their exponentials to offload the MUFU
- * unit (range reduction to n + f, f in [-1/2, 1/2], degree-3 minimax
- * polynomial for 2^f; relative error <= 1.1e-4 for x >= -64, inputs below -64
- * are treated as -64).
- * x, y: device fp32 arrays of n elements, 16-byte aligned, n >= 0.
- * Exposed so that the approximation's error bound can be tested on the GPU.
- */
-int fattn_exp2_poly(const float* x, float* y, long long n, fattn_stream_t stream);
 
 /* Static, human-readable text for a status code. */
 const char* fattn_status_string(int status);

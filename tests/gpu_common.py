@@ -13,32 +13,51 @@ LSE_MAX_ABS = 1e-3
 GRAD_REL = 2e-2
 
 
-def check_o(o_gpu, o_ref, what=""):
-    """O max-abs <= 1e-2 and mean-abs <= 1e-3.  The max-abs bound is on the
-    computation: O is delivered as bf16, and the rounding of the result itself
-    to that format (half an ulp, <= 2^-8 |O|; 0.0156 at |O| = 4) comes on top."""
+def o_max_abs_bound(o_ref):
+    """The O max-abs bound, element by element: 1e-2, plus -- only where |O_ref| >= 2
+    -- the rounding of the bf16 output itself.  O is delivered as bf16, and a
+    correctly rounded bf16 value lies up to half an ulp (2^-8 |O| at most) from
+    the exact one: 0.0039 below |O| = 2, which the 1e-2 absorbs, but 0.0078 for
+    |O| in [2, 4) and more than 1e-2 from |O| = 4 up.  On the stated workloads
+    |O| stays below 2 almost everywhere, so there the bound is the plain 1e-2."""
+    a = np.abs(o_ref)
+    return O_MAX_ABS + np.where(a >= 2.0, 2.0 ** -8 * a, 0.0)
+
+
+def check_o(o_gpu, o_ref, what="", quiet=False):
+    """O max-abs <= 1e-2 (see o_max_abs_bound for |O_ref| >= 2) and mean-abs <= 1e-3.
+    Prints the errors, so that a run with -s shows the margin."""
     err = np.abs(to_f64(o_gpu) - o_ref) if isinstance(o_gpu, torch.Tensor) else np.abs(o_gpu - o_ref)
     assert np.isfinite(err).all(), f"{what} O has non-finite values"
-    excess = err - (O_MAX_ABS + 2.0 ** -8 * np.abs(o_ref))
-    assert excess.max() <= 0, f"{what} O max-abs {err.max():.3e} (above 1e-2 + 2^-8|O| by {excess.max():.3e})"
+    excess = err - o_max_abs_bound(o_ref)
+    assert excess.max() <= 0, f"{what} O max-abs {err.max():.3e} (above its bound by {excess.max():.3e})"
     assert err.mean() <= O_MEAN_ABS, f"{what} O mean-abs {err.mean():.3e}"
+    n_big = int((np.abs(o_ref) >= 2.0).sum())
+    if not quiet:
+        print(f"[parity] {what} O max-abs {err.max():.3e} mean-abs {err.mean():.3e}"
+              f" (|O_ref| >= 2 at {n_big} of {err.size})")
     return float(err.max()), float(err.mean())
 
 
-def check_lse(lse_gpu, lse_ref, what=""):
+def check_lse(lse_gpu, lse_ref, what="", quiet=False):
     g = lse_gpu.double().cpu().numpy() if isinstance(lse_gpu, torch.Tensor) else lse_gpu
     err = np.abs(g - lse_ref)
     assert np.isfinite(err).all(), f"{what} LSE has non-finite values"
     assert err.max() <= LSE_MAX_ABS, f"{what} LSE max-abs {err.max():.3e}"
+    if not quiet:
+        print(f"[parity] {what} LSE max-abs {err.max():.3e}")
     return float(err.max())
 
 
-def check_grad(g_gpu, g_ref, name, what=""):
+def check_grad(g_gpu, g_ref, name, what="", quiet=False):
     g = to_f64(g_gpu) if isinstance(g_gpu, torch.Tensor) else g_gpu
     err = np.abs(g - g_ref)
     bound = GRAD_REL * np.abs(g_ref).max()
     assert np.isfinite(err).all(), f"{what} {name} has non-finite values"
     assert err.max() <= bound, f"{what} {name} max-abs {err.max():.3e} > {bound:.3e}"
+    if not quiet:
+        print(f"[parity] {what} {name} max-abs {err.max():.3e} = {err.max() / max(np.abs(g_ref).max(), 1e-30):.2e}"
+              " of max|ref|")
     return float(err.max() / max(np.abs(g_ref).max(), 1e-30))
 
 

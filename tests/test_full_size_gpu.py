@@ -52,29 +52,35 @@ def _check_workload(w, full_heads):
     for (b, h) in full_heads:
         qh, kh, vh = (to_f64(t[b, h]) for t in (q, k, v))
         o_ref, lse_ref = oracle.ref_fwd(qh[None, None], kh[None, None], vh[None, None], w.causal, w.scale)
-        check_o(to_f64(o[b, h]), o_ref[0, 0], f"head ({b},{h})")
-        check_lse(lse[b, h], lse_ref[0, 0], f"head ({b},{h})")
+        check_o(to_f64(o[b, h]), o_ref[0, 0], f"{w.name} head ({b},{h})")
+        check_lse(lse[b, h], lse_ref[0, 0], f"{w.name} head ({b},{h})")
         if grads is not None:
             doh = to_f64(do[b, h])
             refs = oracle.ref_bwd_head(qh, kh, vh, doh, w.causal, w.scale)
             dq_max_ref = max(dq_max_ref, float(np.abs(refs[0]).max()))
             for g, r, n in zip(grads, refs, ("dQ", "dK", "dV")):
-                check_grad(to_f64(g[b, h]), r, n, f"head ({b},{h})")
+                check_grad(to_f64(g[b, h]), r, n, f"{w.name} head ({b},{h})")
     rng = np.random.default_rng(w.seed)
+    o_max, o_sum, o_cnt, lse_max, dq_rel = 0.0, 0.0, 0, 0.0, 0.0
     # every head: sampled rows of O, LSE (and dQ)
     for b in range(w.B):
         for h in range(w.H):
             rows = _sampled_rows(w.N, rng)
             qh, kh, vh = (to_f64(t[b, h]) for t in (q, k, v))
             o_r, l_r = oracle.ref_fwd_rows(qh, kh, vh, rows, w.causal, w.scale)
-            check_o(to_f64(o[b, h, rows]), o_r, f"head ({b},{h}) rows")
-            check_lse(lse[b, h, rows], l_r, f"head ({b},{h}) rows")
+            emax, emean = check_o(to_f64(o[b, h, rows]), o_r, f"head ({b},{h}) rows", quiet=True)
+            o_max, o_sum, o_cnt = max(o_max, emax), o_sum + emean * o_r.size, o_cnt + o_r.size
+            lse_max = max(lse_max, check_lse(lse[b, h, rows], l_r, f"head ({b},{h}) rows", quiet=True))
             if grads is not None:
                 doh = to_f64(do[b, h])
                 dq_r = oracle.ref_dq_rows(qh, kh, vh, doh, rows, w.causal, w.scale)
                 err = np.abs(to_f64(grads[0][b, h, rows]) - dq_r).max()
                 bound = 2e-2 * max(dq_max_ref, float(np.abs(dq_r).max()))
                 assert err <= bound, f"dQ rows head ({b},{h}): {err:.3e} > {bound:.3e}"
+                dq_rel = max(dq_rel, err / bound * 2e-2)
+    print(f"[parity] {w.name} sampled rows of all {w.B * w.H} heads: O max-abs {o_max:.3e} mean-abs "
+          f"{o_sum / o_cnt:.3e}, LSE max-abs {lse_max:.3e}" +
+          (f", dQ max-abs {dq_rel:.2e} of the max|ref| bound" if grads is not None else ""))
     # every head: column-sum invariants of the backward.  bf16 rounding of the
     # individual rows makes the sums inexact, so they are bounded relative to the
     # sum of magnitudes (a gross error -- a dropped term, a wrong mask -- breaks this).

@@ -87,6 +87,27 @@ def test_unusual_scales(scale):
                 assert torch.count_nonzero(g).item() == 0
 
 
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("N", [100, 200, 1000])
+@pytest.mark.parametrize("scale", [0.0, -0.2])
+def test_unusual_scales_ragged(scale, N, causal):
+    """Zero and negative scales on sequence lengths with a ragged last tile: the
+    keys past N must get weight 0 even where scale * (masked score) is 0 * inf."""
+    (q, k, v, do), (qg, kg, vg, dog) = gpu_inputs(1, 2, N, 64, 24)
+    o, lse = binding.fwd(qg, kg, vg, causal=causal, scale=scale)
+    dq, dk, dv = binding.bwd(qg, kg, vg, o, lse, dog, causal=causal, scale=scale)
+    assert_device_ok()
+    qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = oracle.ref_fwd(qf, kf, vf, causal, scale)
+    _check_o_derived(o, o_ref, vf)
+    check_lse(lse, lse_ref)
+    for g, r, n in zip((dq, dk, dv), oracle.ref_bwd(qf, kf, vf, dof, causal, scale), "QKV"):
+        if n == "V" or scale != 0.0:
+            check_grad(g, r, "d" + n)
+        else:  # scale 0: dQ = dK = 0 exactly
+            assert torch.count_nonzero(g).item() == 0
+
+
 def test_repeated_calls_are_identical():
     _, (qg, kg, vg, dog) = gpu_inputs(2, 2, 512, 128, 22)
     o1, l1 = binding.fwd(qg, kg, vg, causal=True)
