@@ -7,6 +7,17 @@ Python binding never import it; the two share no code.  See
 """
 from .attention_fp64 import (  # noqa: F401
     brute_fwd,
+    brute_fwd_general,
+    dropout_multiplier,
+    dropout_threshold,
+    finite_diff_grads_general,
+    kv_head_of,
+    philox4x32_10,
+    ref_bwd_general,
+    ref_dq_general_rows,
+    ref_fwd_general,
+    ref_fwd_general_rows,
+    softmax_rows_masked,
     causal_keep,
     finite_diff_grads,
     ref_bwd,

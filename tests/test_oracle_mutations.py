@@ -8,6 +8,7 @@ import pytest
 
 from oracle import attention_fp64 as A
 import test_oracle as pins
+import test_oracle_general as gpins
 
 
 def _softmax_no_norm(s):
@@ -45,7 +46,18 @@ MUTATIONS = [
      lambda: pins.test_ref_bwd_matches_finite_differences(False)),
     ("softmax gradient row term dropped", "softmax_grad", lambda p, dp: p * dp,
      lambda: pins.test_backward_column_sums(True)),
+    ("causal mask aligned top-left", "causal_keep",
+     lambda rows, n, offset=0: np.arange(n)[None, :] <= np.asarray(rows)[:, None],
+     lambda: gpins.test_general_fwd_matches_brute_force(1, 2, 2, 3, 7, 4, True, 0.0)),
+    ("key/value head by modulo", "kv_head_of", lambda h, H, H_kv: h % H_kv,
+     lambda: gpins.test_general_fwd_matches_brute_force(1, 4, 2, 7, 3, 3, False, 0.0)),
+    ("dropout kept weights not rescaled", "dropout_multiplier",
+     lambda bh, rows, n_k, p, seed, offset: (_orig_mult(bh, rows, n_k, p, seed, offset) > 0).astype(float),
+     lambda: gpins.test_dropped_output_is_unbiased()),
+    ("rows with no visible key left undefined", "softmax_rows_masked", A.softmax_rows,
+     lambda: gpins.test_general_fwd_matches_brute_force(1, 4, 2, 7, 3, 3, True, 0.0)),
 ]
+_orig_mult = A.dropout_multiplier
 
 
 @pytest.mark.parametrize("name,attr,repl,pin", MUTATIONS, ids=[m[0] for m in MUTATIONS])
