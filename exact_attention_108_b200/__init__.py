@@ -10,8 +10,10 @@ and a missing library is a hard error (there is no fallback path).
 from .binding import (  # noqa: F401
     FattnError,
     bwd,
+    bwd_ex,
     device_status,
     fwd,
+    fwd_ex,
     load,
     status_string,
     workspace_size,

@@ -27,7 +27,31 @@ NOALLOC_SCRATCH_BYTES = 32 << 20  # FATTN_NOALLOC_SCRATCH_BYTES
 # Every symbol include/fattn.h declares (checked by the CPU test suite).
 EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_bwd_preprocess",
             "fattn_bwd_dkdv", "fattn_bwd_dq", "fattn_status_string", "fattn_last_cuda_error",
-            "fattn_device_status", "fattn_version", "fattn_bwd_noalloc")
+            "fattn_device_status", "fattn_version", "fattn_bwd_noalloc", "fattn_fwd_ex",
+            "fattn_bwd_ex", "fattn_bwd_ex_workspace_size")
+
+
+class FwdParams(ctypes.Structure):
+    """fattn_fwd_params (include/fattn.h)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N_q", ctypes.c_int),
+                ("N_k", ctypes.c_int), ("d", ctypes.c_int), ("causal", ctypes.c_int),
+                ("scale", ctypes.c_float), ("dropout_p", ctypes.c_float),
+                ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+
+
+class BwdParams(ctypes.Structure):
+    """fattn_bwd_params (include/fattn.h)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("dout", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N_q", ctypes.c_int),
+                ("N_k", ctypes.c_int), ("d", ctypes.c_int), ("causal", ctypes.c_int),
+                ("scale", ctypes.c_float), ("dropout_p", ctypes.c_float),
+                ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint),
+                ("deterministic", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 _lib = None
 
@@ -70,6 +94,12 @@ def load():
     L.fattn_last_cuda_error.restype = ctypes.c_char_p
     L.fattn_device_status.argtypes = [i]
     L.fattn_device_status.restype = i
+    L.fattn_fwd_ex.argtypes = [ctypes.POINTER(FwdParams), vp]
+    L.fattn_fwd_ex.restype = i
+    L.fattn_bwd_ex.argtypes = [ctypes.POINTER(BwdParams), vp]
+    L.fattn_bwd_ex.restype = i
+    L.fattn_bwd_ex_workspace_size.argtypes = [ctypes.POINTER(BwdParams)]
+    L.fattn_bwd_ex_workspace_size.restype = sz
     L.fattn_version.argtypes = []
     L.fattn_version.restype = i
     _lib = L
@@ -221,4 +251,64 @@ def bwd_noalloc(q, k, v, o, lse, do, causal: bool = False, scale: float | None =
                                   B, H, N, d, 1 if causal else 0, float(scale), _stream_handle(stream))
     if rc != FATTN_OK:
         raise FattnError(rc, "fattn_bwd_noalloc")
+    return dq, dk, dv
+
+
+def _shapes_general(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    B, H, N_q, d = (int(x) for x in q.shape)
+    Bk, H_kv, N_k, dk_ = (int(x) for x in k.shape)
+    if Bk != B or dk_ != d or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"k and v must be [B, H_kv, N_k, d] with B={B}, d={d}")
+    return B, H, H_kv, N_q, N_k, d
+
+
+def fwd_ex(q, k, v, causal: bool = False, scale: float | None = None, dropout_p: float = 0.0,
+           seed: int = 0, offset: int = 0, out=None, lse=None, stream=None):
+    """General forward (fattn_fwd_ex): q [B,H,N_q,d] against k, v [B,H_kv,N_k,d], causal mask
+    aligned at the bottom right, optional dropout; returns (O, LSE)."""
+    B, H, H_kv, N_q, N_k, d = _shapes_general(q, k, v)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N_q), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check(out, "out")
+    _check(lse, "lse", torch.float32)
+    p = FwdParams(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                  B, H, H_kv, N_q, N_k, d, 1 if causal else 0, float(scale), float(dropout_p),
+                  int(seed), int(offset))
+    rc = load().fattn_fwd_ex(ctypes.byref(p), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_fwd_ex")
+    return out, lse
+
+
+def bwd_ex(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, dropout_p: float = 0.0,
+           seed: int = 0, offset: int = 0, deterministic: bool = False, dq=None, dk=None, dv=None,
+           workspace=None, stream=None):
+    """General backward (fattn_bwd_ex) for the forward of fwd_ex; returns (dQ, dK, dV)."""
+    B, H, H_kv, N_q, N_k, d = _shapes_general(q, k, v)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n)
+    _check(lse, "lse", torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    p = BwdParams(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                  dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N_q, N_k, d,
+                  1 if causal else 0, float(scale), float(dropout_p), int(seed), int(offset),
+                  1 if deterministic else 0, None, 0)
+    need = int(load().fattn_bwd_ex_workspace_size(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    p.workspace = workspace.data_ptr()
+    p.workspace_bytes = _nbytes(workspace)
+    rc = load().fattn_bwd_ex(ctypes.byref(p), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_bwd_ex")
     return dq, dk, dv

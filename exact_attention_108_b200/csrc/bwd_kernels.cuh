@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(256) fattn_bwd_pre_kernel(const __nv_bfloat16*
                                                             float* __restrict__ lse2, float* __restrict__ dq_acc,
                                                             long long heads, int N, int NP) {
   // One thread group per row of the padded statistics [heads][NP]: rows n < N get
-  // D = sum(dO o O) and LSE * log2(e) and have their dQ accumulator row zeroed;
+  // D = sum(dO o O) and LSE * log2(e) and have their dQ accumulator row zeroed
+  // (a row whose LSE is -inf -- no visible key -- has O = 0 and D = 0);
   // the padding rows of a ragged last tile get 0 (finite, and masked where used).
   constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
   constexpr int RPB = 256 / TPR;
@@ -65,9 +66,11 @@ __global__ void __launch_bounds__(256) fattn_bwd_pre_kernel(const __nv_bfloat16*
       acc = fmaf(fa.x, fb.x, acc);
       acc = fmaf(fa.y, fb.y, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + off);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dq_acc) {  // null for the deterministic backward, which has no accumulator
+      float4* z = reinterpret_cast<float4*>(dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int w = TPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
@@ -99,16 +102,29 @@ __global__ void __launch_bounds__(256) fattn_bwd_dq_kernel(const float* __restri
 struct BwdArgs {
   const float* lse2;  // [B*H][stat_stride]  LSE * log2(e)
   const float* dvec;  // [B*H][stat_stride]  D
-  float* dq_acc;      // [B*H*N, D] fp32
-  int N;
-  int num_tiles;      // ceil(N / 128)
-  int stat_stride;    // num_tiles * 128: one head's padded statistics
-  int n_tail;         // rows of the last 128-row tile, 1..128
+  float* dq_acc;      // [B*H*N_q, D] fp32 (unused without the dQ product)
+  int N_q;
+  int num_q_tiles;    // ceil(N_q / 128)
+  int num_kv_tiles;   // ceil(N_k / 128)
+  int stat_stride;    // num_q_tiles * 128: one head's padded statistics
+  int q_tail;         // queries in the last 128-row query tile, 1..128
+  int kv_tail;        // keys in the last 128-row key tile, 1..128
+  int causal_off;     // N_k - N_q: query i sees keys j <= i + causal_off (causal)
+  int G;              // query heads per key/value head (H / H_kv)
   int group_big;      // causal order: heads in each of the first num_big_groups groups;
   int num_big_groups; //   the remaining groups hold group_big - 1 heads
   float scale;        // for dK
   float scale_log2;   // scale * log2(e)
+  sm100::Dropout drop;  // used by the DROPOUT instances only
 };
+
+// First query tile that sees key tile t (causal: query i sees key 128 t iff
+// i >= 128 t - off); every key is seen by the last query, so it is < num_q_tiles.
+__host__ __device__ inline int bwd_first_q_tile(int t, int off, bool causal) {
+  if (!causal) return 0;
+  const int first_row = 128 * t - off;
+  return first_row <= 0 ? 0 : first_row / 128;
+}
 
 template <int D>
 struct BwdCfg {
@@ -164,7 +180,7 @@ enum : int {
 // drain and dP_{i+1}, and dV_{i+1} overlaps the dS arithmetic.  Splitting each
 // row's queries over two warpgroups halves the exponential and dS work on that
 // chain.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT, bool WITH_DQ>
 __global__ void __launch_bounds__(384, 1)
     fattn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -196,16 +212,18 @@ __global__ void __launch_bounds__(384, 1)
     if (threadIdx.x == 0) atomicCAS(&g_fattn_status, 0, kSiteBwdAlign);
     return;
   }
-  const int NT = args.num_tiles;
-  // Non-causal: the key tile varies fastest, so the CTAs resident at one time add
-  // into the same head's dQ rows (which then stay in L2).  Causal: a key tile's
-  // work falls with its index (tile t sees NT - t query tiles), so the heads form
-  // groups of group_big or group_big - 1 and inside a group the longest tiles of
-  // all its heads come first; CTAs start in block order as SMs free up, which
-  // makes this longest-first list scheduling within an L2-sized set of heads.
-  int bh, kv_tile;
+  const int NT = args.num_q_tiles;
+  const int NKT = args.num_kv_tiles;
+  // One CTA per (key/value head, key tile).  Non-causal: the key tile varies
+  // fastest, so the CTAs resident at one time add into the same heads' dQ rows
+  // (which then stay in L2).  Causal: a key tile's work falls with its index, so
+  // the heads form groups of group_big or group_big - 1 and inside a group the
+  // longest tiles of all its heads come first; CTAs start in block order as SMs
+  // free up, which makes this longest-first list scheduling within an L2-sized
+  // set of heads.
+  int bh, kv_tile;  // bh: flattened key/value head b * H_kv + hk
   if (CAUSAL) {
-    const int big = args.group_big, ubig = NT * big, nbig_units = args.num_big_groups * ubig;
+    const int big = args.group_big, ubig = NKT * big, nbig_units = args.num_big_groups * ubig;
     const int u = (int)blockIdx.x;
     int r, hg, h0;
     if (u < nbig_units) {
@@ -214,7 +232,7 @@ __global__ void __launch_bounds__(384, 1)
       hg = big;
       h0 = g * big;
     } else {
-      const int gs = NT * (big - 1), u2 = u - nbig_units, g = u2 / gs;
+      const int gs = NKT * (big - 1), u2 = u - nbig_units, g = u2 / gs;
       r = u2 - g * gs;
       hg = big - 1;
       h0 = args.num_big_groups * big + g * (big - 1);
@@ -222,12 +240,16 @@ __global__ void __launch_bounds__(384, 1)
     bh = h0 + r % hg;
     kv_tile = r / hg;
   } else {
-    bh = (int)(blockIdx.x / (unsigned)NT);
-    kv_tile = (int)(blockIdx.x % (unsigned)NT);
+    bh = (int)(blockIdx.x / (unsigned)NKT);
+    kv_tile = (int)(blockIdx.x % (unsigned)NKT);
   }
-  const int head_row0 = bh * args.N;
-  const int i_begin = CAUSAL ? kv_tile : 0;  // first query tile that sees this key tile
-  const int n_it = NT - i_begin;
+  // Steps: the G query heads that share this key/value head, one after the other,
+  // each over its query tiles i_begin .. NT - 1 (those that see this key tile).
+  const int i_begin = bwd_first_q_tile(kv_tile, args.causal_off, CAUSAL);
+  const int n_head = NT - i_begin;
+  const int n_it = args.G * n_head;
+  auto q_head_of = [&](int it) { return bh * args.G + it / n_head; };   // b*H + h
+  auto q_tile_of = [&](int it) { return i_begin + it % n_head; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
@@ -277,13 +299,13 @@ __global__ void __launch_bounds__(384, 1)
         for (; it < n_it; ++it) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_q_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
-          const int q_tile = i_begin + it;
-          const size_t stat_row = (size_t)bh * args.stat_stride + q_tile * 128;
+          const int q_tile = q_tile_of(it), qh = q_head_of(it);
+          const size_t stat_row = (size_t)qh * args.stat_stride + q_tile * 128;
           mbar_arrive_expect_tx(bar_q_full(s), 2 * C::TILE + 1024);
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb) {
-            tma_load_3d(sQ(s) + kb * C::BLK, &tm_q, bar_q_full(s), kb * 64, q_tile * 128, bh);
-            tma_load_3d(sDO(s) + kb * C::BLK, &tm_do, bar_q_full(s), kb * 64, q_tile * 128, bh);
+            tma_load_3d(sQ(s) + kb * C::BLK, &tm_q, bar_q_full(s), kb * 64, q_tile * 128, qh);
+            tma_load_3d(sDO(s) + kb * C::BLK, &tm_do, bar_q_full(s), kb * 64, q_tile * 128, qh);
           }
           bulk_load(sStat(s), args.lse2 + stat_row, 512, bar_q_full(s));
           bulk_load(sStat(s) + 512, args.dvec + stat_row, 512, bar_q_full(s));
@@ -349,15 +371,17 @@ __global__ void __launch_bounds__(384, 1)
               mma_ts(tmem + C::TM_DK, tA + (kk >> 2) * 64 + 32 + (kk & 3) * 8, db + kk * (2048 >> 4), id_kv,
                      (it > 0 || kk > 0) ? 1u : 0u);
           }
-          // (the Q/dO stage is released by the dQ drain, which reuses it as staging)
-          // dQ^T = K^T dS^T into region B (dP^T already read)
-          {
+          if constexpr (WITH_DQ) {
+            // (the Q/dO stage is released by the dQ drain, which reuses it as staging)
+            // dQ^T = K^T dS^T into region B (dP^T already read)
             const uint64_t da = sdesc_sw128(opaque_u32(sK), kt_lbo), db = sdesc_sw128(opaque_u32(sDS), C::BLK);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tB, da + kk * (2048 >> 4), db + kk * (2048 >> 4), id_q, kk > 0 ? 1u : 0u);
+            mma_commit(bar_dq_full);
+          } else {
+            mma_commit(bar_q_empty(s));  // dV_i and dK_i were the stage's last readers
           }
-          mma_commit(bar_dq_full);
           if (it + 1 < n_it) {
             const int s1 = (it + 1) % C::NS;
             if (!(ok = mbar_wait(bar_q_full(s1), ((it + 1) / C::NS) & 1, abort_flag, kSiteBwdMmaQ))) break;
@@ -366,9 +390,12 @@ __global__ void __launch_bounds__(384, 1)
             // issued before it, and tcgen05.mma of one thread executes in order
             issue_kxq(tA, sK, sQ(s1));
             mma_commit(bar_s_full);
-            // dP^T_{i+1} over region B once dQ^T_i has been drained
-            if (!(ok = mbar_wait(bar_dq_free, it & 1, abort_flag, kSiteBwdMmaDQ))) break;
-            tc_fence_after();
+            // dP^T_{i+1} over region B once dQ^T_i has been drained (without the dQ
+            // product, once dP^T_i was read: the gradient warps did so before ds_full)
+            if constexpr (WITH_DQ) {
+              if (!(ok = mbar_wait(bar_dq_free, it & 1, abort_flag, kSiteBwdMmaDQ))) break;
+              tc_fence_after();
+            }
             issue_kxq(tB, sV, sDO(s1));
             mma_commit(bar_dp_full);
           }
@@ -384,14 +411,14 @@ __global__ void __launch_bounds__(384, 1)
       // i's Q/dO stage; one TMA bulk reduce-add puts it into the accumulator rows,
       // which are contiguous.  The stage goes back to the producer once the reduce
       // has read it, without holding up a gradient warp meanwhile.
-      if (lane == 0) {
+      if (WITH_DQ && lane == 0) {
         for (int it = 0; it < n_it; ++it) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
           // only the tile's rows inside the sequence (a ragged last tile has fewer)
-          const int q_tile = i_begin + it;
-          const int rows = q_tile == NT - 1 ? args.n_tail : 128;
-          float* dst = args.dq_acc + (size_t)(head_row0 + q_tile * 128) * D;
+          const int q_tile = q_tile_of(it);
+          const int rows = q_tile == NT - 1 ? args.q_tail : 128;
+          float* dst = args.dq_acc + ((size_t)q_head_of(it) * args.N_q + q_tile * 128) * D;
           bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows * D * 4));
           bulk_commit();
           bulk_wait_read0();
@@ -420,14 +447,39 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float* lse_s = stat(s) + 64 * h;
       const float* dvec_s = stat(s) + 128 + 64 * h;
-      const bool diag = CAUSAL && it == 0;  // queries c < r of the diagonal tile are masked
-      // P = 0 outside the window lo <= c < hi of this half's 64 queries: on the
-      // diagonal tile the queries before this thread's key, in a ragged last query
-      // tile the queries past the sequence, and everything for a key past it
-      const int q_valid = i_begin + it == NT - 1 ? args.n_tail - 64 * h : 64;
-      const bool k_out = kv_tile == NT - 1 && r >= args.n_tail;
-      const int lo = diag ? r - 64 * h : 0;
+      const int q_tile = q_tile_of(it);
+      // P = 0 outside the window lo <= c < hi of this half's 64 queries.  Causal:
+      // query 128 q_tile + 64 h + c sees key 128 kv_tile + r iff c >= lo, lo =
+      // 128 (kv_tile - q_tile) - off - 64 h + r (> 0 only near the diagonal).  In a
+      // ragged last query tile the queries past the sequence, and for a key past
+      // the sequence every query, are outside too.
+      const int q_valid = q_tile == NT - 1 ? args.q_tail - 64 * h : 64;
+      const bool k_out = kv_tile == NKT - 1 && r >= args.kv_tail;
+      const int lo = CAUSAL ? 128 * (kv_tile - q_tile) - args.causal_off - 64 * h + r : 0;
       const int hi = k_out ? 0 : q_valid;
+      // Dropout: bit c of keep = keep bit of (query 128 q_tile + 64 h + c, this key).
+      // One generator call gives four consecutive keys of one query -- the keys of
+      // the four lanes of a quad -- so each lane of a quad draws every fourth query
+      // (16 calls) and the quad swaps the bits with four shuffles.
+      uint64_t keep = ~0ull;
+      if constexpr (DROPOUT) {
+        const int m = lane & 3;
+        const uint32_t j4 = (uint32_t)(kv_tile * 128 + r) >> 2;  // the same for the whole quad
+        const uint32_t i0 = (uint32_t)(q_tile * 128 + 64 * h);
+        const uint32_t qh = (uint32_t)q_head_of(it);
+        uint64_t mine = 0;  // bits 4t .. 4t+3: keys of the quad, query i0 + 4t + m
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          mine |= (uint64_t)dropout_keep4(args.drop, qh, i0 + 4 * t + m, j4) << (4 * t);
+        keep = 0;
+#pragma unroll
+        for (int src = 0; src < 4; ++src) {  // queries i0 + 4t + src come from quad lane src
+          const uint64_t x = __shfl_sync(0xffffffffu, mine, (lane & ~3) | src) >> m;
+#pragma unroll
+          for (int t = 0; t < 16; ++t) keep |= ((x >> (4 * t)) & 1ull) << (4 * t + src);
+        }
+      }
+      auto zf = [&](int c) { return ((keep >> c) & 1ull) ? args.drop.scale_keep : 0.f; };
       const bool any_mask = __any_sync(0xffffffffu, lo > 0 || hi < 64);  // warp-uniform
       // P^T row, this warpgroup's 64 queries: kept in fp32 for dS, packed to bf16 for dV
       float p[64];
@@ -462,8 +514,13 @@ __global__ void __launch_bounds__(384, 1)
       }
       {
         uint32_t pk[32];
+        if constexpr (DROPOUT) {  // dV takes the dropped, rescaled weights
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) pk[c >> 1] = pack_bf16x2(p[c], p[c + 1]);
+          for (int c = 0; c < 64; c += 2) pk[c >> 1] = pack_bf16x2(p[c] * zf(c), p[c + 1] * zf(c + 1));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) pk[c >> 1] = pack_bf16x2(p[c], p[c + 1]);
+        }
         // bf16 pairs into columns 64h .. 64h+31: inside this warpgroup's own S^T
         // columns, which the other warpgroup never reads
         tmem_st32(tA + 64 * h, pk);
@@ -480,6 +537,10 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t dv[32];
         tmem_ld32(tB + 64 * h + c2 * 32, dv);
         tmem_ld_wait(dv);
+        if constexpr (DROPOUT) {  // dP = (dO V^T) o Z
+#pragma unroll
+          for (int t = 0; t < 32; ++t) dv[t] = __float_as_uint(__uint_as_float(dv[t]) * zf(c2 * 32 + t));
+        }
         uint32_t dsk[16];
 #pragma unroll
         for (int t = 0; t < 16; t += 2) {
@@ -491,15 +552,18 @@ __global__ void __launch_bounds__(384, 1)
                                    p[c + 3] * (__uint_as_float(dv[2 * t + 3]) - d4.w));
         }
         tmem_st16(tA + 64 * h + 32 + c2 * 16, dsk);  // columns 64h+32 .. 64h+63
+        if constexpr (WITH_DQ) {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)  // 16-byte chunk c2*4+q4 of the 64-query block h
-          st_shared_v4(sDS + h * C::BLK + sw128_offset(r, c2 * 4 + q4), dsk[q4 * 4], dsk[q4 * 4 + 1],
-                       dsk[q4 * 4 + 2], dsk[q4 * 4 + 3]);
+          for (int q4 = 0; q4 < 4; ++q4)  // 16-byte chunk c2*4+q4 of the 64-query block h
+            st_shared_v4(sDS + h * C::BLK + sw128_offset(r, c2 * 4 + q4), dsk[q4 * 4], dsk[q4 * 4 + 1],
+                         dsk[q4 * 4 + 2], dsk[q4 * 4 + 3]);
+        }
       }
       tmem_st_wait();
-      fence_async_shared();
+      if constexpr (WITH_DQ) fence_async_shared();
       tc_fence_before();
       mbar_arrive(bar_ds_full);
+      if constexpr (!WITH_DQ) continue;
       // dQ^T_i, this warpgroup's 64 queries -> shared memory as row-major fp32
       // [128 queries][D] in this step's Q/dO stage (free: its last readers, dV_i and
       // dK_i, completed before dQ^T_i) for the reducer's bulk reduce-add

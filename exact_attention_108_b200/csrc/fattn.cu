@@ -1,6 +1,7 @@
 // fattn.cu -- C ABI of libfattn (declared in include/fattn.h): argument
 // validation, TMA tensor-map encoding and kernel launches.  Everything the
-// operation computes runs in the kernels of fwd_kernel.cuh / bwd_kernels.cuh.
+// operation computes runs in the kernels of fwd_kernel.cuh, bwd_kernels.cuh and
+// dq_kernel.cuh.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -13,6 +14,7 @@
 #include "fattn.h"
 
 #include "bwd_kernels.cuh"
+#include "dq_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -75,12 +77,43 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Sequence length rounded up to whole 128-row tiles.
 long long padded_n(int N) { return ((long long)N + 127) / 128 * 128; }
 
-int check_shape(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1) return FATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FATTN_ERR_UNSUPPORTED;
+// One attention problem, as every entry point describes it: B batches of H query
+// heads (N_q rows each) against H_kv key/value heads (N_k rows each), head dim d.
+struct Problem {
+  int B, H, H_kv, N_q, N_k, d, causal;
+  float scale, dropout_p;
+  unsigned long long seed;
+  unsigned int offset;
+  long long q_heads() const { return (long long)B * H; }
+  long long kv_heads() const { return (long long)B * H_kv; }
+};
+
+Problem square(int B, int H, int N, int d, int causal, float scale) {
+  return Problem{B, H, H, N, N, d, causal, scale, 0.f, 0ull, 0u};
+}
+
+int check_problem(const Problem& p) {
+  if (p.B < 1 || p.H < 1 || p.H_kv < 1 || p.N_q < 1 || p.N_k < 1) return FATTN_ERR_INVALID_ARG;
+  if (p.H % p.H_kv != 0) return FATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(p.scale)) return FATTN_ERR_INVALID_ARG;
+  if (p.causal != 0 && p.causal != 1) return FATTN_ERR_INVALID_ARG;
+  if (!(p.dropout_p >= 0.f && p.dropout_p < 1.f)) return FATTN_ERR_INVALID_ARG;  // NaN fails too
+  if (p.d != 64 && p.d != 128) return FATTN_ERR_UNSUPPORTED;
   // rows, and rows rounded up to whole tiles per head, are counted in int
-  if ((long long)B * H * padded_n(N) >= (1ll << 31)) return FATTN_ERR_UNSUPPORTED;
+  if (p.q_heads() * padded_n(p.N_q) >= (1ll << 31) || p.kv_heads() * padded_n(p.N_k) >= (1ll << 31))
+    return FATTN_ERR_UNSUPPORTED;
   return FATTN_OK;
+}
+
+fattn::sm100::Dropout dropout_of(const Problem& p) {
+  fattn::sm100::Dropout d;
+  const double t = std::floor((double)p.dropout_p * 4294967296.0);
+  d.threshold = t >= 4294967295.0 ? 0xFFFFFFFFu : (uint32_t)t;
+  d.scale_keep = (float)(1.0 / (1.0 - (double)p.dropout_p));
+  d.seed_lo = (uint32_t)(p.seed & 0xFFFFFFFFull);
+  d.seed_hi = (uint32_t)(p.seed >> 32);
+  d.offset = p.offset;
+  return d;
 }
 
 template <class K>
@@ -192,10 +225,10 @@ int sched_slot(SchedPool& pool, cudaStream_t st) {
   return -1;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROP>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fattn::FwdArgs& a,
                cudaStream_t st) {
-  auto kern = fattn::fattn_fwd_kernel<D, CAUSAL>;
+  auto kern = fattn::fattn_fwd_kernel<D, CAUSAL, DROP>;
   constexpr int smem = fattn::FwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
   int sms = 0, dev = 0;
@@ -205,12 +238,15 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   fattn::FwdArgs args = a;
   args.sched = nullptr;
   if (CAUSAL) {
-    // forward units: pairs of query tiles; pair p needs min(2p + 2, NT) key tiles,
-    // and a head's keys and values take 4*N*d bytes
-    const long long nt = a.num_q_tiles, np = (nt + 1) / 2;
+    // forward units: pairs of query tiles, each costing the key tiles of its second
+    // tile; a head's keys and values take 4*N_k*d bytes
+    const int nt = a.num_q_tiles, np = (nt + 1) / 2;
     long long work = 0;
-    for (long long p = 0; p < np; ++p) work += (2 * p + 2 < nt ? 2 * p + 2 : nt);
-    causal_groups(a.num_units / (int)np, work, nt, 4ll * a.N * D, sms, &args.group_big, &args.num_big_groups);
+    for (int p = 0; p < np; ++p)
+      work += fattn::fwd_kv_tiles(2 * p + 1 < nt ? 2 * p + 1 : nt - 1, a.num_kv_tiles, a.causal_off, true);
+    const long long longest = fattn::fwd_kv_tiles(nt - 1, a.num_kv_tiles, a.causal_off, true);
+    causal_groups(a.num_units / np, work, longest, 4ll * a.num_kv_tiles * 128 * D, sms, &args.group_big,
+                  &args.num_big_groups);
   }
   SchedPool& pool = g_sched_pool[dev];
   std::unique_lock<std::mutex> lock(pool.mu, std::defer_lock);
@@ -234,92 +270,213 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int D, bool CAUSAL>
-int launch_dkdv(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                const CUtensorMap& mdk, const CUtensorMap& mdv, const fattn::BwdArgs& a, int BH, cudaStream_t st) {
-  auto kern = fattn::fattn_bwd_dkdv_kernel<D, CAUSAL>;
+template <int D>
+int fwd_dispatch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fattn::FwdArgs& a,
+                 bool causal, bool drop, cudaStream_t st) {
+  if (causal)
+    return drop ? launch_fwd<D, true, true>(mq, mk, mv, a, st) : launch_fwd<D, true, false>(mq, mk, mv, a, st);
+  return drop ? launch_fwd<D, false, true>(mq, mk, mv, a, st) : launch_fwd<D, false, false>(mq, mk, mv, a, st);
+}
+
+// The forward of a validated problem (pointers checked by the caller).
+int run_fwd(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (int rc = make_head_map(&mq, q, p.q_heads(), p.N_q, p.d)) return rc;
+  if (int rc = make_head_map(&mk, k, p.kv_heads(), p.N_k, p.d)) return rc;
+  if (int rc = make_head_map(&mv, v, p.kv_heads(), p.N_k, p.d)) return rc;
+  fattn::FwdArgs a;
+  a.lse = lse;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.N_q = p.N_q;
+  a.num_q_tiles = (p.N_q + 127) / 128;
+  a.num_kv_tiles = (p.N_k + 127) / 128;
+  a.kv_tail = p.N_k - (a.num_kv_tiles - 1) * 128;
+  a.causal_off = p.N_k - p.N_q;
+  a.G = p.H / p.H_kv;
+  a.num_units = (int)(p.q_heads() * ((a.num_q_tiles + 1) / 2));
+  a.group_big = 1;
+  a.num_big_groups = 1;
+  a.sched = nullptr;
+  a.scale_log2 = p.scale * kLog2e;
+  a.drop = dropout_of(p);
+  const bool drop = p.dropout_p > 0.f;
+  return p.d == 64 ? fwd_dispatch<64>(mq, mk, mv, a, p.causal, drop, st)
+                   : fwd_dispatch<128>(mq, mk, mv, a, p.causal, drop, st);
+}
+
+// ------------------------------------------------------------------ backward
+template <int D, bool CAUSAL, bool DROP, bool WITH_DQ>
+int launch_dkdv(const CUtensorMap* m, const fattn::BwdArgs& a, long long kv_heads, cudaStream_t st) {
+  auto kern = fattn::fattn_bwd_dkdv_kernel<D, CAUSAL, DROP, WITH_DQ>;
   constexpr int smem = fattn::BwdCfg<D>::SMEM;
   if (int rc = set_smem(kern, smem)) return rc;
-  dim3 grid((unsigned)((long long)BH * a.num_tiles));
+  dim3 grid((unsigned)(kv_heads * a.num_kv_tiles));
   fattn::BwdArgs args = a;
   args.group_big = 1;
-  args.num_big_groups = BH;
+  args.num_big_groups = (int)kv_heads;
   if (CAUSAL) {
-    // units: key tiles; tile t meets NT - t query tiles.  Per head the group
-    // keeps the fp32 dQ accumulator, Q and dO in L2: 8*N*d bytes.
+    // units: key tiles; tile t meets G * (NT - first query tile) query tiles.  Per
+    // key/value head the group keeps the fp32 dQ accumulator, Q and dO of its query
+    // heads in L2: about 8*N_q*d*G bytes.
     int sms = 0;
     if (int rc = sm_count(&sms)) return rc;
-    const long long nt = a.num_tiles;
-    causal_groups(BH, nt * (nt + 1) / 2, nt, 8ll * a.N * D, sms, &args.group_big, &args.num_big_groups);
+    long long work = 0, longest = 0;
+    for (int t = 0; t < a.num_kv_tiles; ++t) {
+      const long long n = (long long)a.G * (a.num_q_tiles - fattn::bwd_first_q_tile(t, a.causal_off, true));
+      work += n;
+      longest = n > longest ? n : longest;
+    }
+    causal_groups((int)kv_heads, work, longest, 8ll * a.num_q_tiles * 128 * D * a.G, sms, &args.group_big,
+                  &args.num_big_groups);
   }
-  kern<<<grid, 384, smem, st>>>(mq, mk, mv, mdo, mdk, mdv, args);
+  kern<<<grid, 384, smem, st>>>(m[0], m[1], m[2], m[3], m[4], m[5], args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dkdv_kernel launch");
+  return FATTN_OK;
+}
+
+template <int D, bool CAUSAL, bool DROP>
+int launch_dq_pass(const CUtensorMap* m, const fattn::DqArgs& a, long long q_heads, cudaStream_t st) {
+  auto kern = fattn::fattn_bwd_dq_pass_kernel<D, CAUSAL, DROP>;
+  constexpr int smem = fattn::DqCfg<D>::SMEM;
+  if (int rc = set_smem(kern, smem)) return rc;
+  dim3 grid((unsigned)(q_heads * a.num_q_tiles));
+  fattn::DqArgs args = a;
+  args.group_big = 1;
+  args.num_big_groups = (int)q_heads;
+  if (CAUSAL) {
+    // units: query tiles; tile t meets fwd_kv_tiles(t) key tiles.  Per query head
+    // the group keeps its keys and values in L2: 4*N_k*d bytes.
+    int sms = 0;
+    if (int rc = sm_count(&sms)) return rc;
+    long long work = 0;
+    for (int t = 0; t < a.num_q_tiles; ++t) work += fattn::fwd_kv_tiles(t, a.num_kv_tiles, a.causal_off, true);
+    const long long longest = fattn::fwd_kv_tiles(a.num_q_tiles - 1, a.num_kv_tiles, a.causal_off, true);
+    causal_groups((int)q_heads, work, longest, 4ll * a.num_kv_tiles * 128 * D, sms, &args.group_big,
+                  &args.num_big_groups);
+  }
+  kern<<<grid, 384, smem, st>>>(m[0], m[1], m[2], m[3], args);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_dq_pass_kernel launch");
   return FATTN_OK;
 }
 
 struct WsParts {
   float* dvec;
   float* lse2;
-  float* dq_acc;
+  float* dq_acc;  // null for the deterministic backward, which needs no accumulator
 };
 
 // Workspace: D and LSE*log2(e) per query row, each head padded to whole 128-row
-// tiles ([B*H][ceil(N/128)*128] fp32, so that every tile's statistics are one
-// aligned 512-byte block), then the fp32 dQ accumulator [B*H*N, d].
-size_t ws_bytes_needed(long long heads, int N, int d) {
-  const size_t stat = align256((size_t)(heads * padded_n(N)) * sizeof(float));
-  return 2 * stat + align256((size_t)heads * N * d * sizeof(float));
+// tiles ([B*H][ceil(N_q/128)*128] fp32, so that every tile's statistics are one
+// aligned 512-byte block), then (default backward only) the fp32 dQ accumulator
+// [B*H*N_q, d].
+size_t ws_bytes_needed(const Problem& p, bool deterministic) {
+  const size_t stat = align256((size_t)(p.q_heads() * padded_n(p.N_q)) * sizeof(float));
+  return 2 * stat + (deterministic ? 0 : align256((size_t)p.q_heads() * p.N_q * p.d * sizeof(float)));
 }
 
-WsParts split_workspace(void* workspace, long long heads, int N) {
+WsParts split_workspace(void* workspace, const Problem& p, bool deterministic) {
   char* ws = static_cast<char*>(workspace);
-  const size_t stat = align256((size_t)(heads * padded_n(N)) * sizeof(float));
-  WsParts p;
-  p.dvec = reinterpret_cast<float*>(ws);
-  p.lse2 = reinterpret_cast<float*>(ws + stat);
-  p.dq_acc = reinterpret_cast<float*>(ws + 2 * stat);
-  return p;
+  const size_t stat = align256((size_t)(p.q_heads() * padded_n(p.N_q)) * sizeof(float));
+  WsParts w;
+  w.dvec = reinterpret_cast<float*>(ws);
+  w.lse2 = reinterpret_cast<float*>(ws + stat);
+  w.dq_acc = deterministic ? nullptr : reinterpret_cast<float*>(ws + 2 * stat);
+  return w;
 }
 
 template <int D>
-int launch_pre(const void* o, const void* dout, const float* lse, long long heads, int N, const WsParts& w,
+int launch_pre(const void* o, const void* dout, const float* lse, const Problem& p, const WsParts& w,
                cudaStream_t st) {
   constexpr int rpb = 256 / (D / 8);
-  const int np = (int)padded_n(N);
-  const long long blocks = (heads * np + rpb - 1) / rpb;
-  fattn::fattn_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                                    static_cast<const __nv_bfloat16*>(dout), lse,
-                                                                    w.dvec, w.lse2, w.dq_acc, heads, N, np);
+  const int np = (int)padded_n(p.N_q);
+  const long long blocks = (p.q_heads() * np + rpb - 1) / rpb;
+  fattn::fattn_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, w.dvec, w.lse2, w.dq_acc,
+      p.q_heads(), p.N_q, np);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fattn_bwd_pre_kernel launch");
   return FATTN_OK;
 }
 
 template <int D>
-int launch_dkdv_d(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
-                  int N, int causal, float scale, const WsParts& w, cudaStream_t st) {
-  const uint64_t heads = (uint64_t)B * H;
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if (int rc = make_head_map(&mq, q, heads, N, D)) return rc;
-  if (int rc = make_head_map(&mdo, dout, heads, N, D)) return rc;
-  if (int rc = make_head_map(&mk, k, heads, N, D)) return rc;
-  if (int rc = make_head_map(&mv, v, heads, N, D)) return rc;
-  if (int rc = make_head_map(&mdk, dk, heads, N, D)) return rc;
-  if (int rc = make_head_map(&mdv, dv, heads, N, D)) return rc;
+int dkdv_dispatch(const CUtensorMap* m, const fattn::BwdArgs& a, long long kv_heads, bool causal, bool drop,
+                  bool with_dq, cudaStream_t st) {
+#define FATTN_DKDV(C, P, W) launch_dkdv<D, C, P, W>(m, a, kv_heads, st)
+  if (causal) {
+    if (drop) return with_dq ? FATTN_DKDV(true, true, true) : FATTN_DKDV(true, true, false);
+    return with_dq ? FATTN_DKDV(true, false, true) : FATTN_DKDV(true, false, false);
+  }
+  if (drop) return with_dq ? FATTN_DKDV(false, true, true) : FATTN_DKDV(false, true, false);
+  return with_dq ? FATTN_DKDV(false, false, true) : FATTN_DKDV(false, false, false);
+#undef FATTN_DKDV
+}
+
+template <int D>
+int dq_pass_dispatch(const CUtensorMap* m, const fattn::DqArgs& a, long long q_heads, bool causal, bool drop,
+                     cudaStream_t st) {
+  if (causal)
+    return drop ? launch_dq_pass<D, true, true>(m, a, q_heads, st) : launch_dq_pass<D, true, false>(m, a, q_heads, st);
+  return drop ? launch_dq_pass<D, false, true>(m, a, q_heads, st) : launch_dq_pass<D, false, false>(m, a, q_heads, st);
+}
+
+// Stage 2 of a validated problem: dK, dV (and, unless deterministic, dS K added
+// into the accumulator).
+int run_dkdv(const Problem& p, const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+             const WsParts& w, bool deterministic, cudaStream_t st) {
+  CUtensorMap m[6];  // q, k, v, dout, dk, dv
+  if (int rc = make_head_map(&m[0], q, p.q_heads(), p.N_q, p.d)) return rc;
+  if (int rc = make_head_map(&m[1], k, p.kv_heads(), p.N_k, p.d)) return rc;
+  if (int rc = make_head_map(&m[2], v, p.kv_heads(), p.N_k, p.d)) return rc;
+  if (int rc = make_head_map(&m[3], dout, p.q_heads(), p.N_q, p.d)) return rc;
+  if (int rc = make_head_map(&m[4], dk, p.kv_heads(), p.N_k, p.d)) return rc;
+  if (int rc = make_head_map(&m[5], dv, p.kv_heads(), p.N_k, p.d)) return rc;
   fattn::BwdArgs a;
   a.lse2 = w.lse2;
   a.dvec = w.dvec;
   a.dq_acc = w.dq_acc;
-  a.N = N;
-  a.num_tiles = (N + 127) / 128;
-  a.stat_stride = (int)padded_n(N);
-  a.n_tail = N - (a.num_tiles - 1) * 128;
-  a.scale = scale;
-  a.scale_log2 = scale * kLog2e;
-  const int BH = B * H;
-  return causal ? launch_dkdv<D, true>(mq, mk, mv, mdo, mdk, mdv, a, BH, st)
-                : launch_dkdv<D, false>(mq, mk, mv, mdo, mdk, mdv, a, BH, st);
+  a.N_q = p.N_q;
+  a.num_q_tiles = (p.N_q + 127) / 128;
+  a.num_kv_tiles = (p.N_k + 127) / 128;
+  a.stat_stride = (int)padded_n(p.N_q);
+  a.q_tail = p.N_q - (a.num_q_tiles - 1) * 128;
+  a.kv_tail = p.N_k - (a.num_kv_tiles - 1) * 128;
+  a.causal_off = p.N_k - p.N_q;
+  a.G = p.H / p.H_kv;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * kLog2e;
+  a.drop = dropout_of(p);
+  const bool drop = p.dropout_p > 0.f;
+  return p.d == 64 ? dkdv_dispatch<64>(m, a, p.kv_heads(), p.causal, drop, !deterministic, st)
+                   : dkdv_dispatch<128>(m, a, p.kv_heads(), p.causal, drop, !deterministic, st);
+}
+
+// The deterministic stage 3: dQ by the separate pass.
+int run_dq_pass(const Problem& p, const void* q, const void* k, const void* v, const void* dout, void* dq,
+                const WsParts& w, cudaStream_t st) {
+  CUtensorMap m[4];  // q, k, v, dout
+  if (int rc = make_head_map(&m[0], q, p.q_heads(), p.N_q, p.d)) return rc;
+  if (int rc = make_head_map(&m[1], k, p.kv_heads(), p.N_k, p.d)) return rc;
+  if (int rc = make_head_map(&m[2], v, p.kv_heads(), p.N_k, p.d)) return rc;
+  if (int rc = make_head_map(&m[3], dout, p.q_heads(), p.N_q, p.d)) return rc;
+  fattn::DqArgs a;
+  a.lse2 = w.lse2;
+  a.dvec = w.dvec;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.N_q = p.N_q;
+  a.num_q_tiles = (p.N_q + 127) / 128;
+  a.num_kv_tiles = (p.N_k + 127) / 128;
+  a.stat_stride = (int)padded_n(p.N_q);
+  a.kv_tail = p.N_k - (a.num_kv_tiles - 1) * 128;
+  a.causal_off = p.N_k - p.N_q;
+  a.G = p.H / p.H_kv;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * kLog2e;
+  a.drop = dropout_of(p);
+  const bool drop = p.dropout_p > 0.f;
+  return p.d == 64 ? dq_pass_dispatch<64>(m, a, p.q_heads(), p.causal, drop, st)
+                   : dq_pass_dispatch<128>(m, a, p.q_heads(), p.causal, drop, st);
 }
 
 template <int D>
@@ -333,30 +490,44 @@ int launch_dq(void* dq, long long rows, float scale, const WsParts& w, cudaStrea
   return FATTN_OK;
 }
 
-int check_workspace(void* workspace, size_t bytes, int B, int H, int N, int d) {
+int check_workspace(void* workspace, size_t bytes, const Problem& p, bool deterministic) {
   if (!workspace) return FATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FATTN_ERR_ALIGNMENT;
-  if (bytes < ws_bytes_needed((long long)B * H, N, d)) return FATTN_ERR_INVALID_ARG;
+  if (bytes < ws_bytes_needed(p, deterministic)) return FATTN_ERR_INVALID_ARG;
   return FATTN_OK;
 }
 
-int check_common(int B, int H, int N, int d, float scale, int causal) {
-  if (!std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return FATTN_ERR_INVALID_ARG;
-  return check_shape(B, H, N, d);
+// The whole backward of a validated problem with checked pointers and workspace.
+int run_bwd(const Problem& p, const void* q, const void* k, const void* v, const void* o, const void* dout,
+            const float* lse, void* dq, void* dk, void* dv, void* workspace, bool deterministic, cudaStream_t st) {
+  const WsParts w = split_workspace(workspace, p, deterministic);
+  if (int rc = p.d == 64 ? launch_pre<64>(o, dout, lse, p, w, st) : launch_pre<128>(o, dout, lse, p, w, st))
+    return rc;
+  if (int rc = run_dkdv(p, q, k, v, dout, dk, dv, w, deterministic, st)) return rc;
+  if (deterministic) return run_dq_pass(p, q, k, v, dout, dq, w, st);
+  const long long rows = p.q_heads() * p.N_q;
+  return p.d == 64 ? launch_dq<64>(dq, rows, p.scale, w, st) : launch_dq<128>(dq, rows, p.scale, w, st);
+}
+
+Problem problem_of(const fattn_fwd_params& x) {
+  return Problem{x.B, x.H, x.H_kv, x.N_q, x.N_k, x.d, x.causal, x.scale, x.dropout_p, x.seed, x.offset};
+}
+Problem problem_of(const fattn_bwd_params& x) {
+  return Problem{x.B, x.H, x.H_kv, x.N_q, x.N_k, x.d, x.causal, x.scale, x.dropout_p, x.seed, x.offset};
 }
 
 }  // namespace
 
 extern "C" {
 
-int fattn_version(void) { return 0x000100; }
+int fattn_version(void) { return 0x000200; }
 
 const char* fattn_status_string(int status) {
   switch (status) {
     case FATTN_OK: return "ok";
     case FATTN_ERR_INVALID_ARG: return "invalid argument";
-    case FATTN_ERR_UNSUPPORTED: return "unsupported shape (need d in {64,128} and B*H*ceil(N/128)*128 < 2^31)";
+    case FATTN_ERR_UNSUPPORTED:
+      return "unsupported shape (need d in {64,128} and B*H*ceil(N_q/128)*128, B*H_kv*ceil(N_k/128)*128 < 2^31)";
     case FATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case FATTN_ERR_CUDA: return "CUDA error (see fattn_last_cuda_error)";
     case FATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";
@@ -383,73 +554,69 @@ int fattn_device_status(int clear) {
 int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
               int causal, float scale, fattn_stream_t stream) {
   if (!q || !k || !v || !o || !lse) return FATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return FATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_shape(B, H, N, d)) return rc;
+  const Problem p = square(B, H, N, d, causal, scale);
+  if (int rc = check_problem(p)) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FATTN_ERR_ALIGNMENT;
+  return run_fwd(p, q, k, v, o, lse, reinterpret_cast<cudaStream_t>(stream));
+}
 
-  const uint64_t heads = (uint64_t)B * H;
-  CUtensorMap mq, mk, mv;
-  if (int rc = make_head_map(&mq, q, heads, N, d)) return rc;
-  if (int rc = make_head_map(&mk, k, heads, N, d)) return rc;
-  if (int rc = make_head_map(&mv, v, heads, N, d)) return rc;
-
-  fattn::FwdArgs a;
-  a.lse = lse;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  a.N = N;
-  a.num_q_tiles = (N + 127) / 128;
-  a.n_tail = N - (a.num_q_tiles - 1) * 128;
-  a.num_units = B * H * ((a.num_q_tiles + 1) / 2);
-  a.group_big = 1;
-  a.num_big_groups = 1;
-  a.sched = nullptr;
-  a.scale_log2 = scale * kLog2e;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) return causal ? launch_fwd<64, true>(mq, mk, mv, a, st) : launch_fwd<64, false>(mq, mk, mv, a, st);
-  return causal ? launch_fwd<128, true>(mq, mk, mv, a, st) : launch_fwd<128, false>(mq, mk, mv, a, st);
+int fattn_fwd_ex(const fattn_fwd_params* x, fattn_stream_t stream) {
+  if (!x || !x->q || !x->k || !x->v || !x->o || !x->lse) return FATTN_ERR_INVALID_ARG;
+  const Problem p = problem_of(*x);
+  if (int rc = check_problem(p)) return rc;
+  if (!aligned16(x->q) || !aligned16(x->k) || !aligned16(x->v) || !aligned16(x->o) || !aligned16(x->lse))
+    return FATTN_ERR_ALIGNMENT;
+  return run_fwd(p, x->q, x->k, x->v, x->o, x->lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {
-  if (check_shape(B, H, N, d) != FATTN_OK) return 0;
-  return ws_bytes_needed((long long)B * H, N, d);
+  const Problem p = square(B, H, N, d, 0, 1.f);
+  if (check_problem(p) != FATTN_OK) return 0;
+  return ws_bytes_needed(p, false);
+}
+
+size_t fattn_bwd_ex_workspace_size(const fattn_bwd_params* x) {
+  if (!x) return 0;
+  const Problem p = problem_of(*x);
+  if (check_problem(p) != FATTN_OK) return 0;
+  return ws_bytes_needed(p, x->deterministic != 0);
 }
 
 int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int B, int H, int N, int d,
                          void* workspace, size_t workspace_bytes, fattn_stream_t stream) {
   if (!o || !dout || !lse || !workspace) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_common(B, H, N, d, 1.f, 0)) return rc;
+  const Problem p = square(B, H, N, d, 0, 1.f);
+  if (int rc = check_problem(p)) return rc;
   if (!aligned16(o) || !aligned16(dout) || !aligned16(lse)) return FATTN_ERR_ALIGNMENT;
-  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
-  const long long heads = (long long)B * H;
-  const WsParts w = split_workspace(workspace, heads, N);
+  if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
+  const WsParts w = split_workspace(workspace, p, false);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_pre<64>(o, dout, lse, heads, N, w, st) : launch_pre<128>(o, dout, lse, heads, N, w, st);
+  return d == 64 ? launch_pre<64>(o, dout, lse, p, w, st) : launch_pre<128>(o, dout, lse, p, w, st);
 }
 
 int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
                    int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
                    fattn_stream_t stream) {
   if (!q || !k || !v || !dout || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_common(B, H, N, d, scale, causal)) return rc;
+  const Problem p = square(B, H, N, d, causal, scale);
+  if (int rc = check_problem(p)) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
     return FATTN_ERR_ALIGNMENT;
-  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
-  const WsParts w = split_workspace(workspace, (long long)B * H, N);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dkdv_d<64>(q, k, v, dout, dk, dv, B, H, N, causal, scale, w, st)
-                 : launch_dkdv_d<128>(q, k, v, dout, dk, dv, B, H, N, causal, scale, w, st);
+  if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
+  const WsParts w = split_workspace(workspace, p, false);
+  return run_dkdv(p, q, k, v, dout, dk, dv, w, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale, void* workspace, size_t workspace_bytes,
                  fattn_stream_t stream) {
   if (!dq || !workspace) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_common(B, H, N, d, scale, 0)) return rc;
+  const Problem p = square(B, H, N, d, 0, scale);
+  if (int rc = check_problem(p)) return rc;
   if (!aligned16(dq)) return FATTN_ERR_ALIGNMENT;
-  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
-  const long long rows = (long long)B * H * N;
-  const WsParts w = split_workspace(workspace, (long long)B * H, N);
+  if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
+  const long long rows = p.q_heads() * N;
+  const WsParts w = split_workspace(workspace, p, false);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? launch_dq<64>(dq, rows, scale, w, st) : launch_dq<128>(dq, rows, scale, w, st);
 }
@@ -458,15 +625,29 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o, const 
               void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale, void* workspace,
               size_t workspace_bytes, fattn_stream_t stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_common(B, H, N, d, scale, causal)) return rc;
+  const Problem p = square(B, H, N, d, causal, scale);
+  if (int rc = check_problem(p)) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FATTN_ERR_ALIGNMENT;
-  if (int rc = check_workspace(workspace, workspace_bytes, B, H, N, d)) return rc;
-  if (int rc = fattn_bwd_preprocess(o, dout, lse, B, H, N, d, workspace, workspace_bytes, stream)) return rc;
-  if (int rc = fattn_bwd_dkdv(q, k, v, dout, dk, dv, B, H, N, d, causal, scale, workspace, workspace_bytes, stream))
-    return rc;
-  return fattn_bwd_dq(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
+  return run_bwd(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fattn_bwd_ex(const fattn_bwd_params* x, fattn_stream_t stream) {
+  if (!x || !x->q || !x->k || !x->v || !x->o || !x->dout || !x->lse || !x->dq || !x->dk || !x->dv ||
+      !x->workspace)
+    return FATTN_ERR_INVALID_ARG;
+  if (x->deterministic != 0 && x->deterministic != 1) return FATTN_ERR_INVALID_ARG;
+  const Problem p = problem_of(*x);
+  if (int rc = check_problem(p)) return rc;
+  if (!aligned16(x->q) || !aligned16(x->k) || !aligned16(x->v) || !aligned16(x->o) || !aligned16(x->dout) ||
+      !aligned16(x->lse) || !aligned16(x->dq) || !aligned16(x->dk) || !aligned16(x->dv))
+    return FATTN_ERR_ALIGNMENT;
+  const bool det = x->deterministic != 0;
+  if (int rc = check_workspace(x->workspace, x->workspace_bytes, p, det)) return rc;
+  return run_bwd(p, x->q, x->k, x->v, x->o, x->dout, x->lse, x->dq, x->dk, x->dv, x->workspace, det,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -504,7 +685,7 @@ int fattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o
                       void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
                       fattn_stream_t stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_common(B, H, N, d, scale, causal)) return rc;
+  if (int rc = check_problem(square(B, H, N, d, causal, scale))) return rc;
   if (fattn_bwd_workspace_size(B, H, N, d) > (size_t)FATTN_NOALLOC_SCRATCH_BYTES) return FATTN_ERR_SCRATCH_TOO_SMALL;
   void* scratch = nullptr;
   if (int rc = noalloc_scratch(&scratch)) return rc;

@@ -43,11 +43,14 @@
 namespace fattn {
 
 struct FwdArgs {
-  float* lse;            // [B*H*N] fp32
-  __nv_bfloat16* o;      // [B*H*N, D] bf16
-  int N;                 // keys (and queries) per head
-  int num_q_tiles;       // ceil(N / 128)
-  int n_tail;            // rows of the last 128-row tile, 1..128
+  float* lse;            // [B*H*N_q] fp32
+  __nv_bfloat16* o;      // [B*H*N_q, D] bf16
+  int N_q;               // queries per head
+  int num_q_tiles;       // ceil(N_q / 128)
+  int num_kv_tiles;      // ceil(N_k / 128)
+  int kv_tail;           // keys in the last 128-key tile, 1..128
+  int causal_off;        // N_k - N_q: query i sees keys j <= i + causal_off (causal)
+  int G;                 // query heads per key/value head (H / H_kv)
   int num_units;         // B*H * ceil(num_q_tiles / 2)
   int group_big;         // causal order: heads in each of the first num_big_groups groups;
   int num_big_groups;    //   the remaining groups hold group_big - 1 heads
@@ -57,7 +60,19 @@ struct FwdArgs {
   // takes units c, c + gridDim.x, ...
   unsigned int* sched;
   float scale_log2;      // scale * log2(e)
+  sm100::Dropout drop;   // used by the DROPOUT instances only
 };
+
+// Key tiles query tile t needs (from tile 0 on): all of them, or, causal, those up to
+// the one holding key 128 t + 127 + off; at least 1 (a tile whose rows see no key
+// still runs once, fully masked, so that its O = 0 and LSE = -inf are written).
+__host__ __device__ inline int fwd_kv_tiles(int t, int nkt, int off, bool causal) {
+  if (!causal) return nkt;
+  const int last = 128 * t + 127 + off;  // last key any row of the tile sees
+  if (last < 0) return 1;
+  const int n = last / 128 + 1;
+  return n < nkt ? n : nkt;
+}
 
 template <int D>
 struct FwdCfg {
@@ -99,7 +114,7 @@ enum : int {  // wait sites recorded in the device status word on a timeout
   kSiteFwdUnit = 0x10a,
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(384, 1)
     fattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -137,10 +152,11 @@ __global__ void __launch_bounds__(384, 1)
   // come first (longest-processing-time order), so the group's short units fill
   // in behind its long ones, while the group's keys and values stay in L2.
   const int NT = args.num_q_tiles;
+  const int NKT = args.num_kv_tiles;
   const int NP = (NT + 1) >> 1;
   const bool dyn = CAUSAL && args.sched != nullptr;
   struct Unit {
-    int bh, head_row0, tile0, n_kv0, n_kv1, n_kv;
+    int bh, kv_bh, head_row0, tile0, n_kv0, n_kv1, n_kv;
   };
   auto unit_of = [&](int u) {
     Unit w;
@@ -166,12 +182,13 @@ __global__ void __launch_bounds__(384, 1)
       pair = u % NP;
     }
     w.bh = bh;
-    w.head_row0 = bh * args.N;
+    w.kv_bh = bh / args.G;  // b*H + h -> b*H_kv + h / G
+    w.head_row0 = bh * args.N_q;
     w.tile0 = 2 * pair;
     const bool has_q1 = w.tile0 + 1 < NT;
     // key tiles each query tile needs (contiguous from 0); 0 = tile absent
-    w.n_kv0 = CAUSAL ? w.tile0 + 1 : NT;
-    w.n_kv1 = has_q1 ? (CAUSAL ? w.tile0 + 2 : NT) : 0;
+    w.n_kv0 = fwd_kv_tiles(w.tile0, NKT, args.causal_off, CAUSAL);
+    w.n_kv1 = has_q1 ? fwd_kv_tiles(w.tile0 + 1, NKT, args.causal_off, CAUSAL) : 0;
     w.n_kv = w.n_kv1 > w.n_kv0 ? w.n_kv1 : w.n_kv0;
     return w;
   };
@@ -245,7 +262,7 @@ __global__ void __launch_bounds__(384, 1)
               const uint32_t dst = sSlot0 + s * C::TILE;
 #pragma unroll
               for (int kb = 0; kb < C::KB; ++kb)
-                tma_load_3d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, j * 128, w.bh);
+                tma_load_3d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, j * 128, w.kv_bh);
               ++it;
               // Q0 after K_0, Q1 after V_0: each into the Q buffer freed longest ago
               if (j == 0 && t < nq) {
@@ -401,11 +418,15 @@ __global__ void __launch_bounds__(384, 1)
         // of the raw scores, turned into the max of scale * score (log2 units); four
         // independent three-input chains keep the dependencies short.
         uint32_t v[4][32];
-        const bool diag_tile = CAUSAL && j == q_tile;
-        // a ragged last key tile: its keys c >= n_tail are past the sequence (their
-        // rows read as zero).  Causal rows never see them: the diagonal mask covers
-        // every key past a valid query.
-        const bool tail_tile = !CAUSAL && j == NT - 1 && args.n_tail < 128;
+        // Keys c >= lim of this tile are masked.  Causal: key 128 j + c is visible to
+        // query 128 q_tile + r iff 128 j + c <= 128 q_tile + r + off, so lim = base + r
+        // with base = 128 (q_tile - j) + off + 1, and only tiles with base < 128
+        // mask anything.  Non-causal: a ragged last key tile, whose keys c >= kv_tail
+        // are past the sequence (their rows read as zero).  Causal rows never see
+        // those: the mask hides every key past N_k from every query before N_q.
+        const int base = 128 * (q_tile - j) + args.causal_off + 1;
+        const bool clip = CAUSAL ? base < 128 : (j == NKT - 1 && args.kv_tail < 128);
+        const int lim = CAUSAL ? base + r : args.kv_tail;
         const float masked = sl2 >= 0.f ? -INFINITY : INFINITY;
         float mx;
         {
@@ -417,15 +438,10 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32(tS + 96, v[3]);
           float pm[4] = {masked, masked, masked, masked};
           auto half = [&](int h) {
-            if (diag_tile) {
+            if (clip) {
   #pragma unroll
               for (int c = h * 64; c < h * 64 + 64; ++c)
-                if (c > r) v[c >> 5][c & 31] = __float_as_uint(masked);
-            }
-            if (tail_tile) {
-  #pragma unroll
-              for (int c = h * 64; c < h * 64 + 64; ++c)
-                if (c >= args.n_tail) v[c >> 5][c & 31] = __float_as_uint(masked);
+                if (c >= lim) v[c >> 5][c & 31] = __float_as_uint(masked);
             }
             if (sl2 >= 0.f) {
   #pragma unroll
@@ -454,7 +470,9 @@ __global__ void __launch_bounds__(384, 1)
         const bool grow = mx > m_ref + kRescaleThreshold;
         if (__any_sync(0xffffffffu, grow)) {
           const float m_new = fmaxf(m_ref, mx);
-          const float alpha = ex2(m_ref - m_new);  // 0 on the first tile (m_ref = -inf)
+          // 0 on a row's first visible keys (m_ref = -inf); 1 where the reference
+          // stays, also while a row has seen no visible key (m_ref = m_new = -inf)
+          const float alpha = m_new == m_ref ? 1.f : ex2(m_ref - m_new);
           l *= alpha;
           m_ref = m_new;
           if (j > 0) {
@@ -472,10 +490,11 @@ __global__ void __launch_bounds__(384, 1)
         // Keys c >= lim of this tile get weight 0, by a select after the exponential:
         // the masked raw scores were set to -inf (+inf for a negative scale), and
         // with scale 0 the product -inf * 0 is NaN, so the exponential alone cannot
-        // be trusted to give 0.  Causal: the diagonal tile, lim = r + 1; otherwise a
-        // ragged last tile, lim = n_tail.
-        const bool clip = CAUSAL ? diag_tile : tail_tile;
-        const int lim = CAUSAL ? r + 1 : args.n_tail;
+        // be trusted to give 0.
+        // Dropout (page 2's op chain: softmax, dropout, then V): the undropped
+        // weights go into the row sum l, the dropped and rescaled ones into P V.
+        uint32_t keep = 0xffffffffu;  // keep bits of the current 32 keys
+        const uint32_t q_row = (uint32_t)(q_tile * 128 + r);
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
         uint32_t pk[2][32];                          // P row as packed bf16 pairs
@@ -492,6 +511,17 @@ __global__ void __launch_bounds__(384, 1)
             p1 = (c + 1 < lim) ? p1 : 0.f;
           }
           acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
+          if constexpr (DROPOUT) {
+            if ((c & 31) == 0) {
+              keep = 0;
+  #pragma unroll
+              for (int u = 0; u < 8; ++u)  // keys c .. c + 31, four per generator call
+                keep |= dropout_keep4(args.drop, (uint32_t)w.bh, q_row, (uint32_t)((j * 128 + c) / 4 + u)) << (4 * u);
+            }
+            const float ks = args.drop.scale_keep;
+            p0 = ((keep >> (c & 31)) & 1u) ? p0 * ks : 0.f;
+            p1 = ((keep >> ((c + 1) & 31)) & 1u) ? p1 * ks : 0.f;
+          }
           pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
         }
         {
@@ -520,8 +550,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(bar_o_free(k));  // O_k may now be overwritten by the next unit
       // O row (bf16) straight to global memory, LSE (natural log) beside it; rows
       // of a ragged last tile past the sequence are not written
-      if (q_tile * 128 + r < args.N) {
-        const float inv_l = 1.f / l;
+      if (q_tile * 128 + r < args.N_q) {
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no visible key: O = 0
         const size_t row = (size_t)(w.head_row0 + q_tile * 128 + r);
         uint4* dst = reinterpret_cast<uint4*>(args.o + row * D);
 #pragma unroll

@@ -336,6 +336,49 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return d;
 }
 
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as
+// 1, 2, 3", SC'11), written from its definition: 10 rounds, each multiplying
+// words 0 and 2 by the round constants (64-bit products split into high and low
+// halves) and mixing
+//   (c0, c1, c2, c3) <- (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)),
+// with the key advanced by the Weyl increments between rounds.
+__device__ __forceinline__ void philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
+                                              uint32_t k1, uint32_t (&out)[4]) {
+#pragma unroll
+  for (int rnd = 0; rnd < 10; ++rnd) {
+    const uint32_t lo0 = 0xD2511F53u * c0, hi0 = __umulhi(0xD2511F53u, c0);
+    const uint32_t lo1 = 0xCD9E8D57u * c2, hi1 = __umulhi(0xCD9E8D57u, c2);
+    c0 = hi1 ^ c1 ^ k0;
+    c1 = lo1;
+    c2 = hi0 ^ c3 ^ k1;
+    c3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+// Dropout of attention weights.  The draw for (head bh, query i, key j) is word
+// j mod 4 of Philox4x32-10 at counter (i, j / 4, bh, offset) with key (seed_lo,
+// seed_hi); the weight is kept iff the draw is >= threshold (= floor(p 2^32)) and
+// then multiplied by scale_keep = 1 / (1 - p).
+struct Dropout {
+  uint32_t threshold;
+  float scale_keep;
+  uint32_t seed_lo, seed_hi, offset;
+};
+
+// Keep bits of keys 4u .. 4u + 3 (bit u of the result for key 4u + u) in row i.
+__device__ __forceinline__ uint32_t dropout_keep4(const Dropout& dp, uint32_t bh, uint32_t i, uint32_t j4) {
+  uint32_t w[4];
+  philox4x32_10(i, j4, bh, dp.offset, dp.seed_lo, dp.seed_hi, w);
+  return (uint32_t)(w[0] >= dp.threshold) | ((uint32_t)(w[1] >= dp.threshold) << 1) |
+         ((uint32_t)(w[2] >= dp.threshold) << 2) | ((uint32_t)(w[3] >= dp.threshold) << 3);
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");

@@ -92,6 +92,42 @@ int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
               fattn_stream_t stream);
 
 /*
+ * General form of the forward.  Beyond fattn_fwd it takes
+ *   - separate query and key lengths: q, o are [B, H, N_q, d], lse is [B, H, N_q];
+ *     k, v are [B, H_kv, N_k, d];
+ *   - grouped key/value heads: H must be a multiple of H_kv, and query head h of
+ *     batch b reads key/value head h / (H / H_kv) of batch b (H_kv = H: one each;
+ *     H_kv = 1: one for all);
+ *   - a causal mask aligned at the bottom right: query i sees keys
+ *     j <= i + N_k - N_q (the queries are the last N_q positions of the sequence).
+ *     A query that sees no key (only when N_q > N_k) gets O = 0 and LSE = -inf;
+ *   - dropout on the attention weights (page 2's op chain puts Dropout between the
+ *     softmax and the product with V): each weight P_ij is kept with probability
+ *     1 - dropout_p and then divided by 1 - dropout_p, or set to 0.  The draw for
+ *     (flattened head b*H + h, query i, key j) is word j mod 4 of Philox4x32-10
+ *     (Salmon et al., SC'11) at counter (i, floor(j / 4), b*H + h, offset) with key
+ *     (seed mod 2^32, floor(seed / 2^32)); the weight is kept iff that word is
+ *     >= floor(dropout_p * 2^32).  LSE is that of the undropped weights, and the
+ *     backward regenerates the same mask from (seed, offset).
+ * Constraints are fattn_fwd's, per length: B*H*ceil(N_q/128)*128 and
+ * B*H_kv*ceil(N_k/128)*128 below 2^31; 0 <= dropout_p < 1.
+ */
+typedef struct fattn_fwd_params {
+  const void* q;   /* [B, H, N_q, d] bf16 */
+  const void* k;   /* [B, H_kv, N_k, d] bf16 */
+  const void* v;   /* [B, H_kv, N_k, d] bf16 */
+  void* o;         /* [B, H, N_q, d] bf16, written */
+  float* lse;      /* [B, H, N_q] fp32, written */
+  int B, H, H_kv, N_q, N_k, d;
+  int causal;      /* 0 or 1 */
+  float scale;
+  float dropout_p; /* 0 = no dropout */
+  unsigned long long seed;
+  unsigned int offset;
+} fattn_fwd_params;
+int fattn_fwd_ex(const fattn_fwd_params* params, fattn_stream_t stream);
+
+/*
  * Bytes of device workspace fattn_bwd needs for this shape (0 for an invalid
  * shape).  Layout inside (each part 256-byte aligned): D [B*H][Np] fp32 and
  * LSE*log2(e) [B*H][Np] fp32, where Np = ceil(N / 128) * 128 (each head padded
@@ -111,6 +147,42 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o,
               const void* dout, const float* lse, void* dq, void* dk, void* dv,
               int B, int H, int N, int d, int causal, float scale,
               void* workspace, size_t workspace_bytes, fattn_stream_t stream);
+
+/*
+ * General form of the backward, for the forward of fattn_fwd_ex: the same
+ * shapes, mask, grouping and dropout arguments (seed and offset must be those of
+ * the forward), plus
+ *   dout [B, H, N_q, d]; dq [B, H, N_q, d]; dk, dv [B, H_kv, N_k, d] (a shared
+ *   key/value head gets the sum over the query heads of its group);
+ *   deterministic: 0 = dQ accumulated with fp32 reduce-adds as in fattn_bwd
+ *     (reproducible only up to the order of those additions); 1 = dQ computed
+ *     by a separate pass that owns each query tile and recomputes S and dP for
+ *     it, so that every output is bit-identical from run to run;
+ *   workspace: device memory of at least fattn_bwd_ex_workspace_size(params)
+ *     bytes, 256-byte aligned (the deterministic backward needs no accumulator).
+ */
+typedef struct fattn_bwd_params {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;      /* the forward's output */
+  const void* dout;   /* dL/dO */
+  const float* lse;   /* the forward's statistic */
+  void* dq;
+  void* dk;
+  void* dv;
+  int B, H, H_kv, N_q, N_k, d;
+  int causal;
+  float scale;
+  float dropout_p;
+  unsigned long long seed;
+  unsigned int offset;
+  int deterministic;
+  void* workspace;
+  size_t workspace_bytes;
+} fattn_bwd_params;
+size_t fattn_bwd_ex_workspace_size(const fattn_bwd_params* params);
+int fattn_bwd_ex(const fattn_bwd_params* params, fattn_stream_t stream);
 
 /*
  * Backward that allocates nothing and takes no workspace argument.
@@ -182,7 +254,7 @@ const char* fattn_last_cuda_error(void);
  */
 int fattn_device_status(int clear);
 
-/* Library version, e.g. 0x000100 for 0.1.0. */
+/* Library version, e.g. 0x000200 for 0.2.0. */
 int fattn_version(void);
 
 #ifdef __cplusplus

@@ -40,7 +40,7 @@ def test_status_strings(lib):
     for s in range(6):
         assert binding.status_string(s)
     assert binding.status_string(0) == "ok"
-    assert lib.fattn_version() == 0x000100
+    assert lib.fattn_version() == 0x000200
 
 
 P = 1 << 20  # a fake, 16-byte aligned "device" address; never dereferenced
@@ -103,3 +103,83 @@ def test_python_binding_rejects_host_tensors():
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         binding.fwd(q, q, q)
+
+
+# ------------------------------------------------------------- general forms
+def test_param_structs_match_the_c_layout(tmp_path):
+    """The ctypes mirrors of fattn_fwd_params / fattn_bwd_params have the C layout
+    (offsets printed by a C program compiled against include/fattn.h)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = {"fattn_fwd_params": binding.FwdParams, "fattn_bwd_params": binding.BwdParams}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "fattn.h"', "int main(void) {"]
+    for cname, py in fields.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'  printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(x.split()[:2]): int(x.split()[2]) for x in out if x}
+    for cname, py in fields.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py)
+        for f, _ in py._fields_:
+            assert got[(cname, f)] == getattr(py, f).offset, (cname, f)
+
+
+def _fwd_ex(lib, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=4, H_kv=2, N_q=100, N_k=300, d=128, causal=1, scale=0.1,
+             dropout_p=0.0, seed=0, offset=0)
+    a.update(kw)
+    p = binding.FwdParams(*[a[f] for f, _ in binding.FwdParams._fields_])
+    return lib.fattn_fwd_ex(ctypes.byref(p), None)
+
+
+def test_fwd_ex_validation(lib):
+    assert lib.fattn_fwd_ex(None, None) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, H_kv=3) == binding.FATTN_ERR_INVALID_ARG      # H not a multiple of H_kv
+    assert _fwd_ex(lib, H_kv=0) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, N_q=0) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, N_k=-1) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, dropout_p=1.0) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, dropout_p=-0.1) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, dropout_p=float("nan")) == binding.FATTN_ERR_INVALID_ARG
+    assert _fwd_ex(lib, d=96) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd_ex(lib, B=1 << 14, H=1 << 10, H_kv=1, N_q=128, N_k=128) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd_ex(lib, B=1 << 14, H=1 << 10, H_kv=1 << 10, N_q=1, N_k=128) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd_ex(lib, v=P + 8) == binding.FATTN_ERR_ALIGNMENT
+    assert _fwd_ex(lib, o=None) == binding.FATTN_ERR_INVALID_ARG
+
+
+def _bwd_params(**kw):
+    a = dict(q=P, k=P, v=P, o=P, dout=P, lse=P, dq=P, dk=P, dv=P, B=2, H=4, H_kv=1, N_q=200, N_k=333, d=64,
+             causal=1, scale=0.1, dropout_p=0.2, seed=7, offset=3, deterministic=0, workspace=P,
+             workspace_bytes=0)
+    a.update(kw)
+    return binding.BwdParams(*[a[f] for f, _ in binding.BwdParams._fields_])
+
+
+def test_bwd_ex_workspace_size_and_validation(lib):
+    def a256(x):
+        return (x + 255) // 256 * 256
+    for det in (0, 1):
+        p = _bwd_params(deterministic=det)
+        stat = a256(2 * 4 * 256 * 4)  # B*H heads, N_q padded to 256 rows
+        acc = 0 if det else a256(2 * 4 * 200 * 64 * 4)
+        assert lib.fattn_bwd_ex_workspace_size(ctypes.byref(p)) == 2 * stat + acc
+    assert lib.fattn_bwd_ex_workspace_size(ctypes.byref(_bwd_params(H_kv=3))) == 0
+    need = lib.fattn_bwd_ex_workspace_size(ctypes.byref(_bwd_params()))
+    assert lib.fattn_bwd_ex(ctypes.byref(_bwd_params(workspace_bytes=need - 1)), None) == binding.FATTN_ERR_INVALID_ARG
+    assert lib.fattn_bwd_ex(ctypes.byref(_bwd_params(workspace_bytes=need, workspace=P + 16)), None) == \
+        binding.FATTN_ERR_ALIGNMENT
+    assert lib.fattn_bwd_ex(ctypes.byref(_bwd_params(workspace_bytes=need, deterministic=2)), None) == \
+        binding.FATTN_ERR_INVALID_ARG
+    assert lib.fattn_bwd_ex(ctypes.byref(_bwd_params(workspace_bytes=need, dq=None)), None) == \
+        binding.FATTN_ERR_INVALID_ARG
+    assert lib.fattn_bwd_ex(None, None) == binding.FATTN_ERR_INVALID_ARG

@@ -1,0 +1,120 @@
+"""GPU parity of the general entry points (fattn_fwd_ex, fattn_bwd_ex) with the fp64
+oracle: separate query and key lengths with the causal mask aligned at the bottom
+right, grouped key/value heads, dropout regenerated from (seed, offset), and the
+deterministic backward (dQ by its own pass)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_108_b200 import binding
+from exact_attention_108_b200.workloads import to_f64
+from gpu_common import assert_device_ok, check_grad, check_o
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, H, H_kv, N_q, N_k, d, seed):
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn((B, H, N_q, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, H_kv, N_k, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, H_kv, N_k, d), generator=g).to(torch.bfloat16)
+    do = torch.randn((B, H, N_q, d), generator=g).to(torch.bfloat16)
+    return (q, k, v, do), tuple(t.cuda() for t in (q, k, v, do))
+
+
+def _check_lse_general(lse, ref, what=""):
+    """LSE max-abs <= 1e-3 where the row sees a key; exactly -inf where it sees none."""
+    g = lse.double().cpu().numpy()
+    empty = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(g), empty), f"{what} rows with no visible key differ"
+    err = np.abs(g[~empty] - ref[~empty])
+    assert np.isfinite(err).all() and (err.size == 0 or err.max() <= 1e-3), f"{what} LSE max-abs {err.max():.3e}"
+
+
+CASES = [
+    # B, H, H_kv, N_q, N_k, d
+    (1, 2, 2, 128, 512, 128),   # fewer queries than keys, whole tiles
+    (2, 4, 1, 1, 4096, 64),     # one query row against many keys, one shared key/value head
+    (1, 4, 2, 300, 1000, 128),  # ragged on both sides, groups of two
+    (1, 2, 1, 512, 128, 64),    # more queries than keys: causal rows 0..383 see nothing
+    (1, 6, 3, 200, 200, 64),    # square, ragged, grouped
+    (2, 2, 2, 77, 333, 128),    # causal offset not a multiple of the tile
+]
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d", CASES)
+def test_general_shapes_match_oracle(B, H, H_kv, N_q, N_k, d, causal):
+    (q, k, v, do), (qg, kg, vg, dog) = _inputs(B, H, H_kv, N_q, N_k, d, 100 + N_q + N_k + H_kv)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=causal, scale=scale)
+    grads = {det: binding.bwd_ex(qg, kg, vg, o, lse, dog, causal=causal, scale=scale, deterministic=det)
+             for det in (False, True)}
+    assert_device_ok()
+    qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = oracle.ref_fwd_general(qf, kf, vf, causal, scale)
+    check_o(o, o_ref)
+    _check_lse_general(lse, lse_ref)
+    refs = oracle.ref_bwd_general(qf, kf, vf, dof, causal, scale)
+    for det, gs in grads.items():
+        for g, r, n in zip(gs, refs, ("dQ", "dK", "dV")):
+            check_grad(g, r, n, "deterministic" if det else "reduce-add")
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("p", [0.1, 0.5])
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d", [(1, 2, 1, 256, 384, 64), (1, 2, 2, 200, 200, 128)])
+def test_dropout_matches_oracle(B, H, H_kv, N_q, N_k, d, p, causal):
+    (q, k, v, do), (qg, kg, vg, dog) = _inputs(B, H, H_kv, N_q, N_k, d, 7)
+    scale, seed, offset = 1.0 / math.sqrt(d), 0x1234_5678_9ABC, 17
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=causal, scale=scale, dropout_p=p, seed=seed, offset=offset)
+    grads = {det: binding.bwd_ex(qg, kg, vg, o, lse, dog, causal=causal, scale=scale, dropout_p=p, seed=seed,
+                                 offset=offset, deterministic=det) for det in (False, True)}
+    assert_device_ok()
+    qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
+    pf = float(np.float32(p))  # the library takes dropout_p as fp32
+    o_ref, lse_ref = oracle.ref_fwd_general(qf, kf, vf, causal, scale, pf, seed, offset)
+    # dropped weights are up to 1/(1-p) times larger, and so is the bf16 rounding of P
+    err = np.abs(to_f64(o) - o_ref)
+    assert err.max() <= 1e-2 / (1 - p) and err.mean() <= 1e-3 / (1 - p), (err.max(), err.mean())
+    _check_lse_general(lse, lse_ref)
+    refs = oracle.ref_bwd_general(qf, kf, vf, dof, causal, scale, pf, seed, offset)
+    for det, gs in grads.items():
+        for g, r, n in zip(gs, refs, ("dQ", "dK", "dV")):
+            check_grad(g, r, n, f"p={p} " + ("deterministic" if det else "reduce-add"))
+
+
+def test_dropout_depends_on_seed_and_offset_only():
+    _, (qg, kg, vg, _) = _inputs(1, 2, 2, 256, 256, 64, 8)
+    a, _ = binding.fwd_ex(qg, kg, vg, dropout_p=0.3, seed=5, offset=0)
+    b, _ = binding.fwd_ex(qg, kg, vg, dropout_p=0.3, seed=5, offset=0)
+    c, _ = binding.fwd_ex(qg, kg, vg, dropout_p=0.3, seed=5, offset=1)
+    d, _ = binding.fwd_ex(qg, kg, vg, dropout_p=0.3, seed=6, offset=0)
+    assert_device_ok()
+    assert torch.equal(a, b)
+    assert not torch.equal(a, c) and not torch.equal(a, d)
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_deterministic_backward_is_bit_identical(causal):
+    _, (qg, kg, vg, dog) = _inputs(2, 4, 2, 640, 640, 128, 9)
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=causal)
+    runs = [binding.bwd_ex(qg, kg, vg, o, lse, dog, causal=causal, deterministic=True) for _ in range(3)]
+    assert_device_ok()
+    for other in runs[1:]:
+        for a, b in zip(runs[0], other):
+            assert torch.equal(a, b)
+
+
+def test_square_general_call_equals_the_plain_entry_points():
+    _, (qg, kg, vg, dog) = _inputs(1, 3, 3, 384, 384, 64, 10)
+    o1, l1 = binding.fwd(qg, kg, vg, causal=True)
+    o2, l2 = binding.fwd_ex(qg, kg, vg, causal=True)
+    g1 = binding.bwd(qg, kg, vg, o1, l1, dog, causal=True)
+    g2 = binding.bwd_ex(qg, kg, vg, o1, l1, dog, causal=True, deterministic=False)
+    assert_device_ok()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])  # dK, dV: same kernel, fixed order
