@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     FattnError,
     bwd,
     bwd_ex,
+    decode,
     device_status,
     fwd,
     fwd_ex,

@@ -28,7 +28,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20  # FATTN_NOALLOC_SCRATCH_BYTES
 EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_bwd_preprocess",
             "fattn_bwd_dkdv", "fattn_bwd_dq", "fattn_status_string", "fattn_last_cuda_error",
             "fattn_device_status", "fattn_version", "fattn_bwd_noalloc", "fattn_fwd_ex",
-            "fattn_bwd_ex", "fattn_bwd_ex_workspace_size")
+            "fattn_bwd_ex", "fattn_bwd_ex_workspace_size", "fattn_decode", "fattn_decode_workspace_size")
 
 
 class FwdParams(ctypes.Structure):
@@ -39,6 +39,16 @@ class FwdParams(ctypes.Structure):
                 ("N_k", ctypes.c_int), ("d", ctypes.c_int), ("causal", ctypes.c_int),
                 ("scale", ctypes.c_float), ("dropout_p", ctypes.c_float),
                 ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+
+
+class DecodeParams(ctypes.Structure):
+    """fattn_decode_params (include/fattn.h)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("H_kv", ctypes.c_int), ("N_q", ctypes.c_int),
+                ("N_k", ctypes.c_int), ("N_k_cap", ctypes.c_int), ("d", ctypes.c_int), ("causal", ctypes.c_int),
+                ("scale", ctypes.c_float), ("num_splits", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 
 class BwdParams(ctypes.Structure):
@@ -100,6 +110,10 @@ def load():
     L.fattn_bwd_ex.restype = i
     L.fattn_bwd_ex_workspace_size.argtypes = [ctypes.POINTER(BwdParams)]
     L.fattn_bwd_ex_workspace_size.restype = sz
+    L.fattn_decode.argtypes = [ctypes.POINTER(DecodeParams), vp]
+    L.fattn_decode.restype = i
+    L.fattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams)]
+    L.fattn_decode_workspace_size.restype = sz
     L.fattn_version.argtypes = []
     L.fattn_version.restype = i
     _lib = L
@@ -312,3 +326,34 @@ def bwd_ex(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None
     if rc != FATTN_OK:
         raise FattnError(rc, "fattn_bwd_ex")
     return dq, dk, dv
+
+
+def decode(q, k_cache, v_cache, n_k: int | None = None, causal: bool = False, scale: float | None = None,
+           num_splits: int = 0, out=None, lse=None, workspace=None, stream=None):
+    """Decoding attention (fattn_decode): q [B,H,N_q,d] against the first n_k rows of each head
+    of the caches k_cache, v_cache [B,H_kv,N_k_cap,d]; returns (O, LSE)."""
+    if q.dim() != 4 or k_cache.dim() != 4 or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("expected q [B,H,N_q,d] and caches [B,H_kv,N_k_cap,d]")
+    B, H, N_q, d = (int(x) for x in q.shape)
+    H_kv, cap = int(k_cache.shape[1]), int(k_cache.shape[2])
+    n_k = cap if n_k is None else int(n_k)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, n)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N_q), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check(out, "out")
+    _check(lse, "lse", torch.float32)
+    p = DecodeParams(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     B, H, H_kv, N_q, n_k, cap, d, 1 if causal else 0, float(scale), int(num_splits), None, 0)
+    need = int(load().fattn_decode_workspace_size(ctypes.byref(p)))
+    if need > 0:
+        if workspace is None:
+            workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = _nbytes(workspace)
+    rc = load().fattn_decode(ctypes.byref(p), _stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_decode")
+    return out, lse

@@ -16,7 +16,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "fattn.cu")
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("fattn.cu", "fwd_kernel.cuh", "bwd_kernels.cuh", "dq_kernel.cuh", "sm100.cuh")]
+DEPS = [os.path.join(PKG, "csrc", f) for f in ("fattn.cu", "fwd_kernel.cuh", "bwd_kernels.cuh", "dq_kernel.cuh", "decode_kernel.cuh", "sm100.cuh")]
 INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(PKG, "libfattn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -14,6 +14,7 @@
 #include "fattn.h"
 
 #include "bwd_kernels.cuh"
+#include "decode_kernel.cuh"
 #include "dq_kernel.cuh"
 #include "fwd_kernel.cuh"
 
@@ -50,14 +51,16 @@ EncodeTiledFn encode_fn() {
 // with 128-byte swizzle: one box is 64 columns of a 128-row tile of one head.
 // Rows past N inside a head read as zero and are never written, so a ragged last
 // tile needs no special copy.
-int make_head_map(CUtensorMap* map, const void* base, uint64_t heads, uint64_t N, int d) {
+// head_rows: rows allocated per head (>= N; a key/value cache may hold more rows
+// than are filled), 0 = N.
+int make_head_map(CUtensorMap* map, const void* base, uint64_t heads, uint64_t N, int d, uint64_t head_rows = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     t_last_cuda_error = "cuTensorMapEncodeTiled entry point not available";
     return FATTN_ERR_CUDA;
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, N, heads};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, N * (cuuint64_t)d * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (head_rows ? head_rows : N) * (cuuint64_t)d * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -509,6 +512,68 @@ int run_bwd(const Problem& p, const void* q, const void* k, const void* v, const
   return p.d == 64 ? launch_dq<64>(dq, rows, p.scale, w, st) : launch_dq<128>(dq, rows, p.scale, w, st);
 }
 
+// ------------------------------------------------------------------ decoding
+struct DecodePlan {
+  int rows, row_tiles, num_kv_tiles, tiles_per_split, splits;
+};
+
+DecodePlan decode_plan(const fattn_decode_params& x, int sms) {
+  DecodePlan pl;
+  pl.rows = (x.H / x.H_kv) * x.N_q;
+  pl.row_tiles = (pl.rows + 127) / 128;
+  pl.num_kv_tiles = (x.N_k + 127) / 128;
+  long long want = x.num_splits;
+  if (want <= 0) {
+    // about four CTAs per SM in all, with at least four key tiles per split
+    const long long units = (long long)x.B * x.H_kv * pl.row_tiles;
+    want = (4ll * sms) / units;
+    const long long most = (pl.num_kv_tiles + 3) / 4;
+    if (want > most) want = most;
+  }
+  if (want < 1) want = 1;
+  if (want > pl.num_kv_tiles) want = pl.num_kv_tiles;
+  pl.tiles_per_split = (int)((pl.num_kv_tiles + want - 1) / want);
+  pl.splits = (pl.num_kv_tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;  // none empty
+  return pl;
+}
+
+int check_decode(const fattn_decode_params& x) {
+  if (x.B < 1 || x.H < 1 || x.H_kv < 1 || x.N_q < 1 || x.N_k < 1) return FATTN_ERR_INVALID_ARG;
+  if (x.H % x.H_kv != 0 || x.N_k_cap < x.N_k) return FATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(x.scale) || (x.causal != 0 && x.causal != 1) || x.num_splits < 0) return FATTN_ERR_INVALID_ARG;
+  if (x.d != 64 && x.d != 128) return FATTN_ERR_UNSUPPORTED;
+  const long long rows = (long long)(x.H / x.H_kv) * x.N_q;
+  if ((long long)x.B * x.H_kv * ((rows + 127) / 128 * 128) >= (1ll << 31) ||
+      (long long)x.B * x.H_kv * padded_n(x.N_k_cap) >= (1ll << 31))
+    return FATTN_ERR_UNSUPPORTED;
+  return FATTN_OK;
+}
+
+size_t decode_ws_bytes(const fattn_decode_params& x, const DecodePlan& pl) {
+  if (pl.splits == 1) return 0;
+  const size_t rows_all = (size_t)pl.splits * x.B * x.H_kv * pl.rows;
+  return align256(rows_all * x.d * sizeof(float)) + align256(rows_all * sizeof(float));
+}
+
+template <int D, bool CAUSAL>
+int launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fattn::DecodeArgs& a,
+                  cudaStream_t st) {
+  auto kern = fattn::fattn_decode_kernel<D, CAUSAL>;
+  constexpr int smem = fattn::DecodeCfg<D>::SMEM;
+  if (int rc = set_smem(kern, smem)) return rc;
+  const unsigned grid = (unsigned)((long long)a.splits * a.kv_heads * a.row_tiles);
+  kern<<<grid, 192, smem, st>>>(mq, mk, mv, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_decode_kernel launch");
+  if (a.splits > 1) {
+    const long long rows = (long long)a.kv_heads * a.rows;
+    fattn::fattn_decode_merge_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fattn_decode_merge_kernel launch");
+  }
+  return FATTN_OK;
+}
+
 Problem problem_of(const fattn_fwd_params& x) {
   return Problem{x.B, x.H, x.H_kv, x.N_q, x.N_k, x.d, x.causal, x.scale, x.dropout_p, x.seed, x.offset};
 }
@@ -648,6 +713,56 @@ int fattn_bwd_ex(const fattn_bwd_params* x, fattn_stream_t stream) {
   if (int rc = check_workspace(x->workspace, x->workspace_bytes, p, det)) return rc;
   return run_bwd(p, x->q, x->k, x->v, x->o, x->dout, x->lse, x->dq, x->dk, x->dv, x->workspace, det,
                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fattn_decode_workspace_size(const fattn_decode_params* x) {
+  if (!x || check_decode(*x) != FATTN_OK) return 0;
+  int sms = 0;
+  if (sm_count(&sms) != FATTN_OK) return 0;
+  return decode_ws_bytes(*x, decode_plan(*x, sms));
+}
+
+int fattn_decode(const fattn_decode_params* x, fattn_stream_t stream) {
+  if (!x || !x->q || !x->k || !x->v || !x->o || !x->lse) return FATTN_ERR_INVALID_ARG;
+  if (int rc = check_decode(*x)) return rc;
+  if (!aligned16(x->q) || !aligned16(x->k) || !aligned16(x->v) || !aligned16(x->o) || !aligned16(x->lse))
+    return FATTN_ERR_ALIGNMENT;
+  int sms = 0;
+  if (int rc = sm_count(&sms)) return rc;
+  const DecodePlan pl = decode_plan(*x, sms);
+  const size_t need = decode_ws_bytes(*x, pl);
+  if (need > 0) {
+    if (!x->workspace || x->workspace_bytes < need) return FATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(x->workspace) & 255u) return FATTN_ERR_ALIGNMENT;
+  }
+  const long long kv_heads = (long long)x->B * x->H_kv;
+  CUtensorMap mq, mk, mv;
+  // q (and o) viewed per key/value head: the G*N_q rows of its query heads are contiguous
+  if (int rc = make_head_map(&mq, x->q, kv_heads, (uint64_t)pl.rows, x->d)) return rc;
+  if (int rc = make_head_map(&mk, x->k, kv_heads, x->N_k, x->d, x->N_k_cap)) return rc;
+  if (int rc = make_head_map(&mv, x->v, kv_heads, x->N_k, x->d, x->N_k_cap)) return rc;
+  fattn::DecodeArgs a;
+  const size_t rows_all = (size_t)pl.splits * kv_heads * pl.rows;
+  a.o_part = need ? static_cast<float*>(x->workspace) : nullptr;
+  a.lse_part = need ? reinterpret_cast<float*>(static_cast<char*>(x->workspace) +
+                                               align256(rows_all * x->d * sizeof(float)))
+                    : nullptr;
+  a.o = static_cast<__nv_bfloat16*>(x->o);
+  a.lse = x->lse;
+  a.rows = pl.rows;
+  a.row_tiles = pl.row_tiles;
+  a.N_q = x->N_q;
+  a.N_k = x->N_k;
+  a.num_kv_tiles = pl.num_kv_tiles;
+  a.tiles_per_split = pl.tiles_per_split;
+  a.splits = pl.splits;
+  a.kv_heads = (int)kv_heads;
+  a.causal_off = x->N_k - x->N_q;
+  a.scale_log2 = x->scale * kLog2e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (x->d == 64)
+    return x->causal ? launch_decode<64, true>(mq, mk, mv, a, st) : launch_decode<64, false>(mq, mk, mv, a, st);
+  return x->causal ? launch_decode<128, true>(mq, mk, mv, a, st) : launch_decode<128, false>(mq, mk, mv, a, st);
 }
 
 // ---------------------------------------------------------------------------

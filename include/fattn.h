@@ -185,6 +185,43 @@ size_t fattn_bwd_ex_workspace_size(const fattn_bwd_params* params);
 int fattn_bwd_ex(const fattn_bwd_params* params, fattn_stream_t stream);
 
 /*
+ * Attention for incremental decoding: a few new query rows per sequence against
+ * a long key/value cache.  The result is that of fattn_fwd_ex (without dropout);
+ * the work is laid out for this shape instead: the G = H / H_kv query heads that
+ * share a key/value head are packed into one 128-row tile (G * N_q rows; more
+ * rows take more tiles), and the keys of each (key/value head, row tile) are
+ * split into num_splits ranges processed by separate CTAs, whose partial outputs
+ * a second kernel merges by their log-sum-exp.  Page 2 ("落地使用时应关注什么")
+ * separates this incremental inference, bound by reading the cache, from
+ * training.
+ *   q  [B, H, N_q, d] bf16; o [B, H, N_q, d] bf16 and lse [B, H, N_q] fp32, written.
+ *   k, v: the cache, [B, H_kv, N_k_cap, d] bf16 with N_k_cap >= N_k; only the
+ *     first N_k rows of each head are read.
+ *   causal: 1 = query i sees keys j <= i + N_k - N_q (the new rows are the last
+ *     N_q positions of the sequence).
+ *   num_splits: key ranges per (key/value head, row tile); 0 lets the library
+ *     choose (about four CTAs per SM in all); values above ceil(N_k / 128) are
+ *     reduced to it.
+ *   workspace: fattn_decode_workspace_size(params) bytes (0 when one split is
+ *     used), 256-byte aligned; may be null when that size is 0.
+ */
+typedef struct fattn_decode_params {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int B, H, H_kv, N_q, N_k, N_k_cap, d;
+  int causal;
+  float scale;
+  int num_splits;
+  void* workspace;
+  size_t workspace_bytes;
+} fattn_decode_params;
+size_t fattn_decode_workspace_size(const fattn_decode_params* params);
+int fattn_decode(const fattn_decode_params* params, fattn_stream_t stream);
+
+/*
  * Backward that allocates nothing and takes no workspace argument.
  *
  * The pages the library follows have no counterpart of this call.  It is for

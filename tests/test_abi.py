@@ -114,7 +114,8 @@ def test_param_structs_match_the_c_layout(tmp_path):
     cc = shutil.which("gcc") or shutil.which("cc")
     if cc is None:
         pytest.skip("no C compiler")
-    fields = {"fattn_fwd_params": binding.FwdParams, "fattn_bwd_params": binding.BwdParams}
+    fields = {"fattn_fwd_params": binding.FwdParams, "fattn_bwd_params": binding.BwdParams,
+              "fattn_decode_params": binding.DecodeParams}
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "fattn.h"', "int main(void) {"]
     for cname, py in fields.items():
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
@@ -183,3 +184,22 @@ def test_bwd_ex_workspace_size_and_validation(lib):
     assert lib.fattn_bwd_ex(ctypes.byref(_bwd_params(workspace_bytes=need, dq=None)), None) == \
         binding.FATTN_ERR_INVALID_ARG
     assert lib.fattn_bwd_ex(None, None) == binding.FATTN_ERR_INVALID_ARG
+
+
+def _dec(lib, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=2, H=8, H_kv=2, N_q=1, N_k=1000, N_k_cap=1024, d=128, causal=1,
+             scale=0.1, num_splits=0, workspace=None, workspace_bytes=0)
+    a.update(kw)
+    p = binding.DecodeParams(*[a[f] for f, _ in binding.DecodeParams._fields_])
+    return lib.fattn_decode(ctypes.byref(p), None)
+
+
+def test_decode_validation(lib):
+    assert lib.fattn_decode(None, None) == binding.FATTN_ERR_INVALID_ARG
+    assert _dec(lib, N_k_cap=999) == binding.FATTN_ERR_INVALID_ARG    # cache smaller than N_k
+    assert _dec(lib, H_kv=3) == binding.FATTN_ERR_INVALID_ARG
+    assert _dec(lib, num_splits=-1) == binding.FATTN_ERR_INVALID_ARG
+    assert _dec(lib, causal=3) == binding.FATTN_ERR_INVALID_ARG
+    assert _dec(lib, scale=float("inf")) == binding.FATTN_ERR_INVALID_ARG
+    assert _dec(lib, d=32) == binding.FATTN_ERR_UNSUPPORTED
+    assert _dec(lib, q=P + 4) == binding.FATTN_ERR_ALIGNMENT
