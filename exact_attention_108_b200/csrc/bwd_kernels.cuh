@@ -248,8 +248,17 @@ __global__ void __launch_bounds__(384, 1)
   const int i_begin = bwd_first_q_tile(kv_tile, args.causal_off, CAUSAL);
   const int n_head = NT - i_begin;
   const int n_it = args.G * n_head;
-  auto q_head_of = [&](int it) { return bh * args.G + it / n_head; };   // b*H + h
-  auto q_tile_of = [&](int it) { return i_begin + it % n_head; };
+  // step it = g * n_head + qi: query head bh * G + g (= b*H + h), query tile i_begin + qi,
+  // kept as running counters (no division per step)
+  struct Step {
+    int g = 0, qi = 0;
+    __device__ void next(int n) {
+      if (++qi == n) {
+        qi = 0;
+        ++g;
+      }
+    }
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
@@ -279,9 +288,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   // 384 threads launch with 168 registers each (64512 in all): the producer/MMA
-  // warpgroup keeps 56, the other two take 224 (2*128*224 + 128*56 = 64512).
+  // warpgroup keeps 88, the other two take 208 (2*128*208 + 128*88 = 64512); with
+  // 56 for the producer/MMA group its loop state spilled.
   if (warp >= 8) {
-    regs_decrease<56>();
+    regs_decrease<88>();
     if (warp == 8) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {
@@ -296,10 +306,11 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_3d(sV + kb * C::BLK, &tm_v, bar_kv_full, kb * 64, kv_tile * 128, bh);
         }
         int it = 0;
-        for (; it < n_it; ++it) {
+        Step sx;
+        for (; it < n_it; ++it, sx.next(n_head)) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_q_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
-          const int q_tile = q_tile_of(it), qh = q_head_of(it);
+          const int q_tile = i_begin + sx.qi, qh = bh * args.G + sx.g;
           const size_t stat_row = (size_t)qh * args.stat_stride + q_tile * 128;
           mbar_arrive_expect_tx(bar_q_full(s), 2 * C::TILE + 1024);
 #pragma unroll
@@ -412,13 +423,14 @@ __global__ void __launch_bounds__(384, 1)
       // which are contiguous.  The stage goes back to the producer once the reduce
       // has read it, without holding up a gradient warp meanwhile.
       if (WITH_DQ && lane == 0) {
-        for (int it = 0; it < n_it; ++it) {
+        Step sx;
+        for (int it = 0; it < n_it; ++it, sx.next(n_head)) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
           // only the tile's rows inside the sequence (a ragged last tile has fewer)
-          const int q_tile = q_tile_of(it);
+          const int q_tile = i_begin + sx.qi;
           const int rows = q_tile == NT - 1 ? args.q_tail : 128;
-          float* dst = args.dq_acc + ((size_t)q_head_of(it) * args.N_q + q_tile * 128) * D;
+          float* dst = args.dq_acc + ((size_t)(bh * args.G + sx.g) * args.N_q + q_tile * 128) * D;
           bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows * D * 4));
           bulk_commit();
           bulk_wait_read0();
@@ -429,7 +441,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     }
   } else {
-    regs_increase<224>();
+    regs_increase<208>();
     // ---------------------------------------------------------- gradient warps
     const int h = warp >> 2;   // query half: queries 64h .. 64h+63 of each tile
     const int wq = warp & 3;   // TMEM lane quarter of this warp
@@ -439,7 +451,8 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = args.scale_log2;
     const bool has_d = r < D;  // TMEM lane = head-dim index of dQ^T
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+    Step sx;
+    for (int it = 0; it < n_it; ++it, sx.next(n_head)) {
       const int s = it % C::NS;
       ok = mbar_wait(bar_s_full, it & 1, abort_flag, kSiteBwdSoftS);
       ok = ok && mbar_wait(bar_q_full(s), (it / C::NS) & 1, abort_flag, kSiteBwdSoftS);
@@ -447,7 +460,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float* lse_s = stat(s) + 64 * h;
       const float* dvec_s = stat(s) + 128 + 64 * h;
-      const int q_tile = q_tile_of(it);
+      const int q_tile = i_begin + sx.qi;
       // P = 0 outside the window lo <= c < hi of this half's 64 queries.  Causal:
       // query 128 q_tile + 64 h + c sees key 128 kv_tile + r iff c >= lo, lo =
       // 128 (kv_tile - q_tile) - off - 64 h + r (> 0 only near the diagonal).  In a
@@ -466,7 +479,7 @@ __global__ void __launch_bounds__(384, 1)
         const int m = lane & 3;
         const uint32_t j4 = (uint32_t)(kv_tile * 128 + r) >> 2;  // the same for the whole quad
         const uint32_t i0 = (uint32_t)(q_tile * 128 + 64 * h);
-        const uint32_t qh = (uint32_t)q_head_of(it);
+        const uint32_t qh = (uint32_t)(bh * args.G + sx.g);
         uint64_t mine = 0;  // bits 4t .. 4t+3: keys of the quad, query i0 + 4t + m
 #pragma unroll
         for (int t = 0; t < 16; ++t)
