@@ -43,7 +43,10 @@ __global__ void __launch_bounds__(256) fattn_bwd_pre_kernel(const __nv_bfloat16*
   // D = sum(dO o O) and LSE * log2(e) and have their dQ accumulator row zeroed
   // (a row whose LSE is -inf -- no visible key -- has O = 0 and D = 0);
   // the padding rows of a ragged last tile get 0 (finite, and masked where used).
-  constexpr int TPR = D / 8;  // threads per row, 8 elements (16 bytes) each
+  // threads per row, 8-element (16-byte) pieces each: D / 8 of them for d = 64, 128;
+  // 4 for d = 32, 96 (one and three pieces each), so that TPR is a power of two
+  constexpr int TPR = D % 64 == 0 ? D / 8 : 4;
+  constexpr int PIECES = D / (8 * TPR);
   constexpr int RPB = 256 / TPR;
   const long long prow = (long long)blockIdx.x * RPB + threadIdx.x / TPR;
   const bool in_range = prow < heads * NP;
@@ -54,22 +57,25 @@ __global__ void __launch_bounds__(256) fattn_bwd_pre_kernel(const __nv_bfloat16*
   const int part = threadIdx.x % TPR;
   float acc = 0.f;
   if (valid) {
-    const size_t off = (size_t)row * D + part * 8;
-    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
-    const uint4 b = *reinterpret_cast<const uint4*>(dout + off);
-    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 fa = __bfloat1622float2(pa[i]);
-      const float2 fb = __bfloat1622float2(pb[i]);
-      acc = fmaf(fa.x, fb.x, acc);
-      acc = fmaf(fa.y, fb.y, acc);
-    }
-    if (dq_acc) {  // null for the deterministic backward, which has no accumulator
-      float4* z = reinterpret_cast<float4*>(dq_acc + off);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int pc = 0; pc < PIECES; ++pc) {
+      const size_t off = (size_t)row * D + (part * PIECES + pc) * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+      const uint4 b = *reinterpret_cast<const uint4*>(dout + off);
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa = __bfloat1622float2(pa[i]);
+        const float2 fb = __bfloat1622float2(pb[i]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+      if (dq_acc) {  // null for the deterministic backward, which has no accumulator
+        float4* z = reinterpret_cast<float4*>(dq_acc + off);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
 #pragma unroll
@@ -128,10 +134,10 @@ __host__ __device__ inline int bwd_first_q_tile(int t, int off, bool causal) {
 
 template <int D>
 struct BwdCfg {
-  static constexpr int KB = D / 64;            // 64-column (128-byte) blocks per row
+  using L = sm100::Cols<D>;                    // column blocks of a K, V, Q or dO tile
   static constexpr int NS = 2;                 // Q/dO ring depth
   static constexpr int TILE = 128 * D * 2;     // bytes of a 128-row K, V, Q or dO tile
-  static constexpr int BLK = 128 * 128;        // one 64-column block of a 128-row tile
+  static constexpr int DS_BLK = 128 * 128;     // one 64-query block of dS^T (128-byte swizzle)
   static constexpr int DS_BYTES = 128 * 128 * 2;  // dS^T [128 keys][128 queries] bf16
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = TILE;
@@ -301,9 +307,9 @@ __global__ void __launch_bounds__(384, 1)
         prefetch_tensormap(&tm_do);
         mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_3d(sK + kb * C::BLK, &tm_k, bar_kv_full, kb * 64, kv_tile * 128, bh);
-          tma_load_3d(sV + kb * C::BLK, &tm_v, bar_kv_full, kb * 64, kv_tile * 128, bh);
+        for (int kb = 0; kb < C::L::NB; ++kb) {
+          tma_load_3d(sK + kb * C::L::BLKB, &tm_k, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
+          tma_load_3d(sV + kb * C::L::BLKB, &tm_v, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
         }
         int it = 0;
         Step sx;
@@ -314,9 +320,9 @@ __global__ void __launch_bounds__(384, 1)
           const size_t stat_row = (size_t)qh * args.stat_stride + q_tile * 128;
           mbar_arrive_expect_tx(bar_q_full(s), 2 * C::TILE + 1024);
 #pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb) {
-            tma_load_3d(sQ(s) + kb * C::BLK, &tm_q, bar_q_full(s), kb * 64, q_tile * 128, qh);
-            tma_load_3d(sDO(s) + kb * C::BLK, &tm_do, bar_q_full(s), kb * 64, q_tile * 128, qh);
+          for (int kb = 0; kb < C::L::NB; ++kb) {
+            tma_load_3d(sQ(s) + kb * C::L::BLKB, &tm_q, bar_q_full(s), kb * C::L::CW, q_tile * 128, qh);
+            tma_load_3d(sDO(s) + kb * C::L::BLKB, &tm_do, bar_q_full(s), kb * C::L::CW, q_tile * 128, qh);
           }
           bulk_load(sStat(s), args.lse2 + stat_row, 512, bar_q_full(s));
           bulk_load(sStat(s) + 512, args.dvec + stat_row, 512, bar_q_full(s));
@@ -336,7 +342,9 @@ __global__ void __launch_bounds__(384, 1)
         constexpr uint32_t id_q = idesc_bf16_f32(128, 128, true, true);    // K^T (MN) x dS^T (MN)
         // For d = 64 the dQ^T product still uses M = 128: the second 64-row half of
         // A repeats the first (LBO = 0) and its output lanes are ignored.
-        constexpr uint32_t kt_lbo = (D == 128) ? C::BLK : 0;
+        // (d = 32 likewise repeats its one block four times; for d = 96 the fourth
+        // block lies past K, inside the V tile, and only feeds the ignored lanes 96..127)
+        constexpr uint32_t kt_lbo = C::L::NB > 1 ? C::L::BLKB : 0;
         const uint32_t tA = tmem + C::TM_A, tB = tmem + C::TM_B;
         // Descriptors: the start address is a descriptor's low 14 bits (address /
         // 16, below 2^14 for any shared-memory address), so each K step adds a
@@ -344,10 +352,10 @@ __global__ void __launch_bounds__(384, 1)
         // through an opaque move, so that the descriptors of every tile and step
         // are not hoisted out of the loop into this thread's 56 registers.
         auto issue_kxq = [&](uint32_t dst, uint32_t a_tile, uint32_t b_tile) {  // dst = A_tile B_tile^T, K = D
-          const uint64_t da = sdesc_sw128(opaque_u32(a_tile), 16), db = sdesc_sw128(opaque_u32(b_tile), 16);
+          const uint64_t da = C::L::desc_k(opaque_u32(a_tile)), db = C::L::desc_k(opaque_u32(b_tile));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off16 = ((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4;
+            const uint32_t off16 = C::L::kstep(kk) >> 4;
             mma_ss(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
           }
         };
@@ -366,29 +374,30 @@ __global__ void __launch_bounds__(384, 1)
           if (!(ok = mbar_wait(bar_p_full, it & 1, abort_flag, kSiteBwdMmaP))) break;
           tc_fence_after();
           {
-            const uint64_t db = sdesc_sw128(opaque_u32(sDO(s)), C::BLK);
+            const uint64_t db = C::L::desc_mn(opaque_u32(sDO(s)), C::L::BLKB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // queries 16kk..: P^T of half kk/4 at columns 64*(kk/4) + 8*(kk%4)
-              mma_ts(tmem + C::TM_DV, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (2048 >> 4), id_kv,
+              mma_ts(tmem + C::TM_DV, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4), id_kv,
                      (it > 0 || kk > 0) ? 1u : 0u);
           }
           // dK += dS^T Q  (A = dS^T from TMEM, two 64-query halves)
           if (!(ok = mbar_wait(bar_ds_full, it & 1, abort_flag, kSiteBwdMmaDS))) break;
           tc_fence_after();
           {
-            const uint64_t db = sdesc_sw128(opaque_u32(sQ(s)), C::BLK);
+            const uint64_t db = C::L::desc_mn(opaque_u32(sQ(s)), C::L::BLKB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // dS^T of half kk/4 at columns 64*(kk/4) + 32 + 8*(kk%4)
-              mma_ts(tmem + C::TM_DK, tA + (kk >> 2) * 64 + 32 + (kk & 3) * 8, db + kk * (2048 >> 4), id_kv,
+              mma_ts(tmem + C::TM_DK, tA + (kk >> 2) * 64 + 32 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4),
+                     id_kv,
                      (it > 0 || kk > 0) ? 1u : 0u);
           }
           if constexpr (WITH_DQ) {
             // (the Q/dO stage is released by the dQ drain, which reuses it as staging)
             // dQ^T = K^T dS^T into region B (dP^T already read)
-            const uint64_t da = sdesc_sw128(opaque_u32(sK), kt_lbo), db = sdesc_sw128(opaque_u32(sDS), C::BLK);
+            const uint64_t da = C::L::desc_mn(opaque_u32(sK), kt_lbo), db = sdesc_sw128(opaque_u32(sDS), C::DS_BLK);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tB, da + kk * (2048 >> 4), db + kk * (2048 >> 4), id_q, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)  // 16 keys per step: 16 rows of K, 16 rows of dS^T
+              mma_ss(tB, da + kk * (C::L::ROWSTEP16 >> 4), db + kk * (2048 >> 4), id_q, kk > 0 ? 1u : 0u);
             mma_commit(bar_dq_full);
           } else {
             mma_commit(bar_q_empty(s));  // dV_i and dK_i were the stage's last readers
@@ -568,7 +577,7 @@ __global__ void __launch_bounds__(384, 1)
         if constexpr (WITH_DQ) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)  // 16-byte chunk c2*4+q4 of the 64-query block h
-            st_shared_v4(sDS + h * C::BLK + sw128_offset(r, c2 * 4 + q4), dsk[q4 * 4], dsk[q4 * 4 + 1],
+            st_shared_v4(sDS + h * C::DS_BLK + sw128_offset(r, c2 * 4 + q4), dsk[q4 * 4], dsk[q4 * 4 + 1],
                          dsk[q4 * 4 + 2], dsk[q4 * 4 + 3]);
         }
       }
@@ -617,10 +626,10 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld32(tsrc + c * 32, w32);
             tmem_ld_wait(w32);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int chunk = (c & 1) * 4 + q4;
+            for (int q4 = 0; q4 < 4; ++q4) {  // columns c*32 + 8 q4 .. +7: block, then 16-byte chunk in it
+              const int col = c * 32 + q4 * 8;
               const uint32_t* w = &w32[q4 * 8];
-              st_shared_v4(sdst + (c >> 1) * C::BLK + sw128_offset(row, chunk),
+              st_shared_v4(sdst + (col / C::L::CW) * C::L::BLKB + C::L::chunk_offset(row, (col % C::L::CW) / 8),
                            pack_bf16x2(__uint_as_float(w[0]) * mul, __uint_as_float(w[1]) * mul),
                            pack_bf16x2(__uint_as_float(w[2]) * mul, __uint_as_float(w[3]) * mul),
                            pack_bf16x2(__uint_as_float(w[4]) * mul, __uint_as_float(w[5]) * mul),
@@ -632,10 +641,10 @@ __global__ void __launch_bounds__(384, 1)
         named_barrier(1, 128);
         if (wq == 0 && lane == 0) {
 #pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb) {
+          for (int kb = 0; kb < C::L::NB; ++kb) {
             // 3-D stores: rows of a ragged last key tile past the sequence are not written
-            tma_store_3d(&tm_dv, sV + kb * C::BLK, kb * 64, kv_tile * 128, bh);
-            tma_store_3d(&tm_dk, sK + kb * C::BLK, kb * 64, kv_tile * 128, bh);
+            tma_store_3d(&tm_dv, sV + kb * C::L::BLKB, kb * C::L::CW, kv_tile * 128, bh);
+            tma_store_3d(&tm_dk, sK + kb * C::L::BLKB, kb * C::L::CW, kv_tile * 128, bh);
           }
           bulk_commit();
           bulk_wait0();

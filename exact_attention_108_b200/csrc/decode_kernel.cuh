@@ -47,15 +47,14 @@ struct DecodeArgs {
 
 template <int D>
 struct DecodeCfg {
-  static constexpr int KB = D / 64;
+  using L = sm100::Cols<D>;
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int BLK = 128 * 128;
-  static constexpr int NSLOT = (D == 128) ? 6 : 12;
+  static constexpr int NSLOT = D == 128 ? 6 : D == 96 ? 8 : D == 64 ? 12 : 16;
   static constexpr int OFF_Q = 0, OFF_SLOT = TILE;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * TILE;
-  // q_full, slot_full[NSLOT], slot_empty[NSLOT], s_full[2], p_full, pv_done, drain
+  // q_full, slot_full[NSLOT], slot_empty[NSLOT], s_full[2], p_full[2], pv_done, o_done, drain
   static constexpr int B_Q = 0, B_SF = 1, B_SE = 1 + NSLOT, B_S = 1 + 2 * NSLOT, B_P = B_S + 2;
-  static constexpr int B_PV = B_P + 1, B_DRAIN = B_P + 2, NBAR = B_DRAIN + 1;
+  static constexpr int B_PV = B_P + 2, B_OD = B_PV + 1, B_DRAIN = B_PV + 2, NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -89,7 +88,11 @@ __global__ void __launch_bounds__(192, 1)
   auto bar_slot_full = [&](int s) { return bar(C::B_SF + s); };
   auto bar_slot_empty = [&](int s) { return bar(C::B_SE + s); };
   auto bar_s_full = [&](int b) { return bar(C::B_S + b); };
-  const uint32_t bar_p_full = bar(C::B_P), bar_pv_done = bar(C::B_PV), bar_drain = bar(C::B_DRAIN);
+  // p_full has one barrier per S buffer: warps whose rows are all padding pass a tile
+  // at once, and with a single barrier their arrivals for tile j + 1 could complete
+  // tile j's phase before the warp with real rows had written P_j
+  auto bar_p_full = [&](int b) { return bar(C::B_P + b); };
+  const uint32_t bar_pv_done = bar(C::B_PV), bar_o_done = bar(C::B_OD), bar_drain = bar(C::B_DRAIN);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -115,8 +118,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(bar_s_full(0), 1);
     mbar_init(bar_s_full(1), 1);
-    mbar_init(bar_p_full, 128);
+    mbar_init(bar_p_full(0), 128);
+    mbar_init(bar_p_full(1), 128);
     mbar_init(bar_pv_done, 1);
+    mbar_init(bar_o_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -138,7 +143,8 @@ __global__ void __launch_bounds__(192, 1)
       prefetch_tensormap(&tm_v);
       mbar_arrive_expect_tx(bar_q_full, C::TILE);
 #pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb) tma_load_3d(sQ + kb * C::BLK, &tm_q, bar_q_full, kb * 64, rt * 128, hb);
+      for (int kb = 0; kb < C::L::NB; ++kb)
+        tma_load_3d(sQ + kb * C::L::BLKB, &tm_q, bar_q_full, kb * C::L::CW, rt * 128, hb);
       int it = 0;  // K_j at 2j, V_j at 2j + 1 (j counted from the split's first tile)
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
@@ -148,8 +154,9 @@ __global__ void __launch_bounds__(192, 1)
           mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
           const CUtensorMap* map = t == 0 ? &tm_k : &tm_v;
 #pragma unroll
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_3d(sSlot0 + s * C::TILE + kb * C::BLK, map, bar_slot_full(s), kb * 64, (j0 + j) * 128, hb);
+          for (int kb = 0; kb < C::L::NB; ++kb)
+            tma_load_3d(sSlot0 + s * C::TILE + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW,
+                        (j0 + j) * 128, hb);
         }
       }
       if (!ok) {  // aborted: let the copies already issued land before the CTA exits
@@ -169,10 +176,10 @@ __global__ void __launch_bounds__(192, 1)
         return mbar_wait(bar_slot_full(i % C::NSLOT), (i / C::NSLOT) & 1, abort_flag, site);
       };
       auto issue_s = [&](int j) {  // S_j = Q K_j^T into buffer j & 1
-        const uint64_t dq = sdesc_sw128(opaque_u32(sQ), 16), dk = sdesc_sw128(opaque_u32(slot_addr(2 * j)), 16);
+        const uint64_t dq = C::L::desc_k(opaque_u32(sQ)), dk = C::L::desc_k(opaque_u32(slot_addr(2 * j)));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off16 = ((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4;
+          const uint32_t off16 = C::L::kstep(kk) >> 4;
           mma_ss(tmem + C::TM_S + (j & 1) * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_s_full(j & 1));
@@ -186,14 +193,14 @@ __global__ void __launch_bounds__(192, 1)
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         // O += P_j V_j (P_j, bf16, over the first 64 columns of S buffer j & 1)
-        if (!(ok = mbar_wait(bar_p_full, j & 1, abort_flag, kSiteDecMmaP))) break;
+        if (!(ok = mbar_wait(bar_p_full(j & 1), (j >> 1) & 1, abort_flag, kSiteDecMmaP))) break;
         if (!(ok = wait_slot(2 * j + 1, kSiteDecMmaV))) break;
         tc_fence_after();
         const uint32_t tP = tmem + C::TM_S + (j & 1) * 128;
-        const uint64_t dv = sdesc_sw128(opaque_u32(slot_addr(2 * j + 1)), C::BLK);
+        const uint64_t dv = C::L::desc_mn(opaque_u32(slot_addr(2 * j + 1)), C::L::BLKB);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::TM_O, tP + kk * 8, dv + kk * (2048 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::TM_O, tP + kk * 8, dv + kk * (C::L::ROWSTEP16 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_pv_done);
         mma_commit(bar_slot_empty((2 * j + 1) % C::NSLOT));
         // S_{j+2} over buffer j & 1: P_j V_j, issued just before, reads it first
@@ -203,6 +210,7 @@ __global__ void __launch_bounds__(192, 1)
           issue_s(j + 2);
         }
       }
+      if (ok) mma_commit(bar_o_done);  // every P_j V_j is in O
       mma_commit(bar_drain);
       mbar_wait_ns(bar_drain, 0, 100000000ull);
     }
@@ -265,7 +273,9 @@ __global__ void __launch_bounds__(192, 1)
           l *= alpha;
           m_ref = m_new;
           if (j > 0) {
-            // O holds P_{j-1} V_{j-1} once that product is done
+            // O holds P_{j-1} V_{j-1} once that product is done.  The parity wait is
+            // unambiguous: S_j was issued after P_{j-2} V_{j-2}, so that product is done
+            // and pv_done has completed j - 1 or j phases.
             ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done, (j - 1) & 1, abort_flag, kSiteDecSoftO));
             if (!ok) break;
             tc_fence_after();
@@ -307,9 +317,9 @@ __global__ void __launch_bounds__(192, 1)
         tmem_st_wait();
       }
       tc_fence_before();
-      mbar_arrive(bar_p_full);
+      mbar_arrive(bar_p_full(j & 1));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_pv_done, (n_kv - 1) & 1, abort_flag, kSiteDecSoftO));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, 0, abort_flag, kSiteDecSoftO));
     if (ok && warp_live) {
       tc_fence_after();
       uint32_t o[D / 32][32];
@@ -375,8 +385,7 @@ __global__ void __launch_bounds__(256) fattn_decode_merge_kernel(const DecodeArg
   const size_t base = (size_t)hb * args.rows + prow;
   float m = -INFINITY;
   for (int s = 0; s < args.splits; ++s) m = fmaxf(m, args.lse_part[base + s * stride]);
-  constexpr int PER = D / 32;  // 4 or 2 columns per lane
-  static_assert(PER == 4 || PER == 2, "d = 128 or 64");
+  constexpr int PER = D / 32;  // columns per lane: 1 to 4
   float acc[PER] = {};
   float wsum = 0.f;
   if (m != -INFINITY) {
@@ -385,26 +394,14 @@ __global__ void __launch_bounds__(256) fattn_decode_merge_kernel(const DecodeArg
       const float w = sm100::ex2(L - m);  // 0 for a split where the row sees no key
       wsum += w;
       const float* src = args.o_part + (base + s * stride) * D + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] = fmaf(w, x.x, acc[0]);
-        acc[1] = fmaf(w, x.y, acc[1]);
-        acc[2] = fmaf(w, x.z, acc[2]);
-        acc[3] = fmaf(w, x.w, acc[3]);
-      } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        acc[0] = fmaf(w, x.x, acc[0]);
-        acc[1] = fmaf(w, x.y, acc[1]);
-      }
+#pragma unroll
+      for (int c = 0; c < PER; ++c) acc[c] = fmaf(w, src[c], acc[c]);
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   __nv_bfloat16* dst = args.o + ((size_t)hb * args.rows + prow) * D + lane * PER;
-  if constexpr (PER == 4)
-    *reinterpret_cast<uint2*>(dst) = make_uint2(sm100::pack_bf16x2(acc[0] * inv, acc[1] * inv),
-                                                sm100::pack_bf16x2(acc[2] * inv, acc[3] * inv));
-  else
-    *reinterpret_cast<uint32_t*>(dst) = sm100::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+#pragma unroll
+  for (int c = 0; c < PER; ++c) dst[c] = __float2bfloat16_rn(acc[c] * inv);
   if (lane == 0) args.lse[(size_t)hb * args.rows + prow] = (m + __log2f(wsum)) * 0.69314718055994530942f;
 }
 

@@ -16,7 +16,7 @@
 // Roles (384 threads = three warpgroups):
 //   warps 0..7  gradient warps.  Warpgroup h takes keys 64h .. 64h+63 of every
 //               key tile; thread = query row of the tile.  Both write the dQ rows
-//               at the end, warpgroup h the columns h D/2 .. (h+1) D/2 - 1.
+//               at the end, warpgroup h the 32-column chunks c with c % 2 == h.
 //   warp 8      TMA producer: Q_i, dO_i once; K_j, V_j through an NSLOT-deep ring
 //   warp 9      tcgen05 issuer (one thread); warps 10, 11 idle
 // Tensor memory (512 columns): S in two buffers (columns 0 and 128; dS, bf16,
@@ -53,10 +53,9 @@ struct DqArgs {
 
 template <int D>
 struct DqCfg {
-  static constexpr int KB = D / 64;
+  using L = sm100::Cols<D>;
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int BLK = 128 * 128;
-  static constexpr int NSLOT = (D == 128) ? 4 : 6;  // K/V ring
+  static constexpr int NSLOT = D == 128 ? 4 : D == 96 ? 4 : D == 64 ? 6 : 8;  // K/V ring
   static constexpr int OFF_Q = 0, OFF_DO = TILE, OFF_SLOT = 2 * TILE;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * TILE;
   // q_full, slot_full[NSLOT], slot_empty[NSLOT], s_full[2], dp_full, ds_full, done, drain
@@ -175,9 +174,9 @@ __global__ void __launch_bounds__(384, 1)
         prefetch_tensormap(&tm_do);
         mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE);
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_3d(sQ + kb * C::BLK, &tm_q, bar_q_full, kb * 64, q_tile * 128, bh);
-          tma_load_3d(sDO + kb * C::BLK, &tm_do, bar_q_full, kb * 64, q_tile * 128, bh);
+        for (int kb = 0; kb < C::L::NB; ++kb) {
+          tma_load_3d(sQ + kb * C::L::BLKB, &tm_q, bar_q_full, kb * C::L::CW, q_tile * 128, bh);
+          tma_load_3d(sDO + kb * C::L::BLKB, &tm_do, bar_q_full, kb * C::L::CW, q_tile * 128, bh);
         }
         int it = 0;  // tiles loaded: K_j at 2j, V_j at 2j + 1
         bool ok = true;
@@ -189,8 +188,9 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
             const CUtensorMap* map = t == 0 ? &tm_k : &tm_v;
 #pragma unroll
-            for (int kb = 0; kb < C::KB; ++kb)
-              tma_load_3d(sSlot0 + s * C::TILE + kb * C::BLK, map, bar_slot_full(s), kb * 64, j * 128, kv_bh);
+            for (int kb = 0; kb < C::L::NB; ++kb)
+              tma_load_3d(sSlot0 + s * C::TILE + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW, j * 128,
+                          kv_bh);
           }
         }
         if (!ok) {  // aborted: let the copies already issued land before the CTA exits
@@ -211,10 +211,10 @@ __global__ void __launch_bounds__(384, 1)
         };
         // dst = A B^T with K = D, both operands K-major 128-row tiles
         auto issue_rows = [&](uint32_t dst, uint32_t a_tile, uint32_t b_tile) {
-          const uint64_t da = sdesc_sw128(opaque_u32(a_tile), 16), db = sdesc_sw128(opaque_u32(b_tile), 16);
+          const uint64_t da = C::L::desc_k(opaque_u32(a_tile)), db = C::L::desc_k(opaque_u32(b_tile));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off16 = ((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4;
+            const uint32_t off16 = C::L::kstep(kk) >> 4;
             mma_ss(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
           }
         };
@@ -246,10 +246,10 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           {
             const uint32_t tA = tmem + C::TM_S + (j & 1) * 128;
-            const uint64_t db = sdesc_sw128(opaque_u32(slot_addr(kslot)), C::BLK);
+            const uint64_t db = C::L::desc_mn(opaque_u32(slot_addr(kslot)), C::L::BLKB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // keys 16kk..: dS of half kk/4 at columns 64*(kk/4) + 8*(kk%4)
-              mma_ts(tmem + C::TM_DQ, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (2048 >> 4), id_dq,
+              mma_ts(tmem + C::TM_DQ, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4), id_dq,
                      (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar_slot_empty(kslot % C::NSLOT));
@@ -350,29 +350,30 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(bar_ds_full);
     }
-    // dQ rows (thread = query row) -> scale -> bf16 -> global memory; warpgroup h
-    // writes columns h D/2 .. (h+1) D/2 - 1; rows past N_q are not written
+    // dQ rows (thread = query row) -> scale -> bf16 -> global memory, 32 columns at a
+    // time: warpgroup h takes the 32-column chunks c with c % 2 == h; rows past N_q
+    // are not written
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, kSiteDqEpi));
     if (ok) {
       tc_fence_after();
-      uint32_t o[D / 64][32];
+      const bool row_ok = q_tile * 128 + r < args.N_q;
+      const float sc = args.scale;
+      uint4* dst = reinterpret_cast<uint4*>(args.dq + ((size_t)bh * args.N_q + q_tile * 128 + r) * D);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) tmem_ld32(tmem + C::TM_DQ + h * (D / 2) + c * 32 + lane_off, o[c]);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) tmem_ld_wait(o[c]);
-      if (q_tile * 128 + r < args.N_q) {
-        const float sc = args.scale;
-        uint4* dst = reinterpret_cast<uint4*>(args.dq + ((size_t)bh * args.N_q + q_tile * 128 + r) * D + h * (D / 2));
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
+      for (int c = h; c < D / 32; c += 2) {
+        uint32_t o[32];
+        tmem_ld32(tmem + C::TM_DQ + c * 32 + lane_off, o);
+        tmem_ld_wait(o);
+        if (row_ok) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            const uint32_t* x = &o[c][q4 * 8];
+            const uint32_t* x = &o[q4 * 8];
             dst[c * 4 + q4] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * sc, __uint_as_float(x[1]) * sc),
                                          pack_bf16x2(__uint_as_float(x[2]) * sc, __uint_as_float(x[3]) * sc),
                                          pack_bf16x2(__uint_as_float(x[4]) * sc, __uint_as_float(x[5]) * sc),
                                          pack_bf16x2(__uint_as_float(x[6]) * sc, __uint_as_float(x[7]) * sc));
           }
+        }
       }
     }
     tc_fence_before();

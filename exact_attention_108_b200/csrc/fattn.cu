@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "fattn.h"
 
@@ -61,10 +62,14 @@ int make_head_map(CUtensorMap* map, const void* base, uint64_t heads, uint64_t N
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, N, heads};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (head_rows ? head_rows : N) * (cuuint64_t)d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  // 64-column boxes with 128-byte swizzle for d = 64, 128; 32-column boxes with
+  // 64-byte swizzle for d = 32, 96 (a box never reaches past a row)
+  const bool wide = d % 64 == 0;
+  cuuint32_t box[3] = {wide ? 64u : 32u, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, wide ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[96];
@@ -73,6 +78,17 @@ int make_head_map(CUtensorMap* map, const void* base, uint64_t heads, uint64_t N
     return FATTN_ERR_CUDA;
   }
   return FATTN_OK;
+}
+
+// Calls f with the head dim as a compile-time constant (validated: 32, 64, 96 or 128).
+template <class F>
+int by_d(int d, F&& f) {
+  switch (d) {
+    case 32: return f(std::integral_constant<int, 32>{});
+    case 64: return f(std::integral_constant<int, 64>{});
+    case 96: return f(std::integral_constant<int, 96>{});
+    default: return f(std::integral_constant<int, 128>{});
+  }
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -101,7 +117,7 @@ int check_problem(const Problem& p) {
   if (!std::isfinite(p.scale)) return FATTN_ERR_INVALID_ARG;
   if (p.causal != 0 && p.causal != 1) return FATTN_ERR_INVALID_ARG;
   if (!(p.dropout_p >= 0.f && p.dropout_p < 1.f)) return FATTN_ERR_INVALID_ARG;  // NaN fails too
-  if (p.d != 64 && p.d != 128) return FATTN_ERR_UNSUPPORTED;
+  if (p.d != 32 && p.d != 64 && p.d != 96 && p.d != 128) return FATTN_ERR_UNSUPPORTED;
   // rows, and rows rounded up to whole tiles per head, are counted in int
   if (p.q_heads() * padded_n(p.N_q) >= (1ll << 31) || p.kv_heads() * padded_n(p.N_k) >= (1ll << 31))
     return FATTN_ERR_UNSUPPORTED;
@@ -303,8 +319,7 @@ int run_fwd(const Problem& p, const void* q, const void* k, const void* v, void*
   a.scale_log2 = p.scale * kLog2e;
   a.drop = dropout_of(p);
   const bool drop = p.dropout_p > 0.f;
-  return p.d == 64 ? fwd_dispatch<64>(mq, mk, mv, a, p.causal, drop, st)
-                   : fwd_dispatch<128>(mq, mk, mv, a, p.causal, drop, st);
+  return by_d(p.d, [&](auto D) { return fwd_dispatch<D.value>(mq, mk, mv, a, p.causal, drop, st); });
 }
 
 // ------------------------------------------------------------------ backward
@@ -451,8 +466,8 @@ int run_dkdv(const Problem& p, const void* q, const void* k, const void* v, cons
   a.scale_log2 = p.scale * kLog2e;
   a.drop = dropout_of(p);
   const bool drop = p.dropout_p > 0.f;
-  return p.d == 64 ? dkdv_dispatch<64>(m, a, p.kv_heads(), p.causal, drop, !deterministic, st)
-                   : dkdv_dispatch<128>(m, a, p.kv_heads(), p.causal, drop, !deterministic, st);
+  return by_d(p.d,
+              [&](auto D) { return dkdv_dispatch<D.value>(m, a, p.kv_heads(), p.causal, drop, !deterministic, st); });
 }
 
 // The deterministic stage 3: dQ by the separate pass.
@@ -478,8 +493,7 @@ int run_dq_pass(const Problem& p, const void* q, const void* k, const void* v, c
   a.scale_log2 = p.scale * kLog2e;
   a.drop = dropout_of(p);
   const bool drop = p.dropout_p > 0.f;
-  return p.d == 64 ? dq_pass_dispatch<64>(m, a, p.q_heads(), p.causal, drop, st)
-                   : dq_pass_dispatch<128>(m, a, p.q_heads(), p.causal, drop, st);
+  return by_d(p.d, [&](auto D) { return dq_pass_dispatch<D.value>(m, a, p.q_heads(), p.causal, drop, st); });
 }
 
 template <int D>
@@ -504,12 +518,11 @@ int check_workspace(void* workspace, size_t bytes, const Problem& p, bool determ
 int run_bwd(const Problem& p, const void* q, const void* k, const void* v, const void* o, const void* dout,
             const float* lse, void* dq, void* dk, void* dv, void* workspace, bool deterministic, cudaStream_t st) {
   const WsParts w = split_workspace(workspace, p, deterministic);
-  if (int rc = p.d == 64 ? launch_pre<64>(o, dout, lse, p, w, st) : launch_pre<128>(o, dout, lse, p, w, st))
-    return rc;
+  if (int rc = by_d(p.d, [&](auto D) { return launch_pre<D.value>(o, dout, lse, p, w, st); })) return rc;
   if (int rc = run_dkdv(p, q, k, v, dout, dk, dv, w, deterministic, st)) return rc;
   if (deterministic) return run_dq_pass(p, q, k, v, dout, dq, w, st);
   const long long rows = p.q_heads() * p.N_q;
-  return p.d == 64 ? launch_dq<64>(dq, rows, p.scale, w, st) : launch_dq<128>(dq, rows, p.scale, w, st);
+  return by_d(p.d, [&](auto D) { return launch_dq<D.value>(dq, rows, p.scale, w, st); });
 }
 
 // ------------------------------------------------------------------ decoding
@@ -541,7 +554,7 @@ int check_decode(const fattn_decode_params& x) {
   if (x.B < 1 || x.H < 1 || x.H_kv < 1 || x.N_q < 1 || x.N_k < 1) return FATTN_ERR_INVALID_ARG;
   if (x.H % x.H_kv != 0 || x.N_k_cap < x.N_k) return FATTN_ERR_INVALID_ARG;
   if (!std::isfinite(x.scale) || (x.causal != 0 && x.causal != 1) || x.num_splits < 0) return FATTN_ERR_INVALID_ARG;
-  if (x.d != 64 && x.d != 128) return FATTN_ERR_UNSUPPORTED;
+  if (x.d != 32 && x.d != 64 && x.d != 96 && x.d != 128) return FATTN_ERR_UNSUPPORTED;
   const long long rows = (long long)(x.H / x.H_kv) * x.N_q;
   if ((long long)x.B * x.H_kv * ((rows + 127) / 128 * 128) >= (1ll << 31) ||
       (long long)x.B * x.H_kv * padded_n(x.N_k_cap) >= (1ll << 31))
@@ -592,7 +605,7 @@ const char* fattn_status_string(int status) {
     case FATTN_OK: return "ok";
     case FATTN_ERR_INVALID_ARG: return "invalid argument";
     case FATTN_ERR_UNSUPPORTED:
-      return "unsupported shape (need d in {64,128} and B*H*ceil(N_q/128)*128, B*H_kv*ceil(N_k/128)*128 < 2^31)";
+      return "unsupported shape (need d in {32,64,96,128} and B*H*ceil(N_q/128)*128, B*H_kv*ceil(N_k/128)*128 < 2^31)";
     case FATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case FATTN_ERR_CUDA: return "CUDA error (see fattn_last_cuda_error)";
     case FATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";
@@ -657,7 +670,7 @@ int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int 
   if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
   const WsParts w = split_workspace(workspace, p, false);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_pre<64>(o, dout, lse, p, w, st) : launch_pre<128>(o, dout, lse, p, w, st);
+  return by_d(d, [&](auto D) { return launch_pre<D.value>(o, dout, lse, p, w, st); });
 }
 
 int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B, int H,
@@ -683,7 +696,7 @@ int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale, void* worksp
   const long long rows = p.q_heads() * N;
   const WsParts w = split_workspace(workspace, p, false);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_dq<64>(dq, rows, scale, w, st) : launch_dq<128>(dq, rows, scale, w, st);
+  return by_d(d, [&](auto D) { return launch_dq<D.value>(dq, rows, scale, w, st); });
 }
 
 int fattn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
@@ -760,9 +773,9 @@ int fattn_decode(const fattn_decode_params* x, fattn_stream_t stream) {
   a.causal_off = x->N_k - x->N_q;
   a.scale_log2 = x->scale * kLog2e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (x->d == 64)
-    return x->causal ? launch_decode<64, true>(mq, mk, mv, a, st) : launch_decode<64, false>(mq, mk, mv, a, st);
-  return x->causal ? launch_decode<128, true>(mq, mk, mv, a, st) : launch_decode<128, false>(mq, mk, mv, a, st);
+  return by_d(x->d, [&](auto D) {
+    return x->causal ? launch_decode<D.value, true>(mq, mk, mv, a, st) : launch_decode<D.value, false>(mq, mk, mv, a, st);
+  });
 }
 
 // ---------------------------------------------------------------------------

@@ -76,11 +76,10 @@ __host__ __device__ inline int fwd_kv_tiles(int t, int nkt, int off, bool causal
 
 template <int D>
 struct FwdCfg {
-  static constexpr int KB = D / 64;                 // 128-byte column blocks per row
+  using L = sm100::Cols<D>;                         // column blocks of a tile
   static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row Q/K/V tile
-  static constexpr int BLK = 128 * 128;             // one 64-column block of a tile
   static constexpr int QBUF = 3;                    // Q tile ring
-  static constexpr int NSLOT = (D == 128) ? 4 : 6;  // K/V ring depth
+  static constexpr int NSLOT = D == 128 ? 4 : D == 96 ? 6 : D == 64 ? 6 : 8;  // K/V ring depth
   static constexpr int NUNIT = 4;                   // ring of unit indices from the producer
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_SLOT = QBUF * TILE;
@@ -261,8 +260,8 @@ __global__ void __launch_bounds__(384, 1)
               const CUtensorMap* map = (t == 0) ? &tm_k : &tm_v;
               const uint32_t dst = sSlot0 + s * C::TILE;
 #pragma unroll
-              for (int kb = 0; kb < C::KB; ++kb)
-                tma_load_3d(dst + kb * C::BLK, map, bar_slot_full(s), kb * 64, j * 128, w.kv_bh);
+              for (int kb = 0; kb < C::L::NB; ++kb)
+                tma_load_3d(dst + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW, j * 128, w.kv_bh);
               ++it;
               // Q0 after K_0, Q1 after V_0: each into the Q buffer freed longest ago
               if (j == 0 && t < nq) {
@@ -271,8 +270,9 @@ __global__ void __launch_bounds__(384, 1)
                   break;
                 mbar_arrive_expect_tx(bar_q_full(b), C::TILE);
 #pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                  tma_load_3d(sQ(b) + kb * C::BLK, &tm_q, bar_q_full(b), kb * 64, (w.tile0 + t) * 128, w.bh);
+                for (int kb = 0; kb < C::L::NB; ++kb)
+                  tma_load_3d(sQ(b) + kb * C::L::BLKB, &tm_q, bar_q_full(b), kb * C::L::CW, (w.tile0 + t) * 128,
+                              w.bh);
                 ++qs;
               }
             }
@@ -299,11 +299,11 @@ __global__ void __launch_bounds__(384, 1)
           // one base descriptor per operand.  The bases pass through an opaque
           // move: hoisted out of the loops, the descriptors of every buffer and
           // step would not fit in this thread's registers.
-          const uint64_t dq = sdesc_sw128(opaque_u32(sQ(qbuf)), 16);
-          const uint64_t dk = sdesc_sw128(opaque_u32(sSlot0 + kslot * C::TILE), 16);
+          const uint64_t dq = C::L::desc_k(opaque_u32(sQ(qbuf)));
+          const uint64_t dk = C::L::desc_k(opaque_u32(sSlot0 + kslot * C::TILE));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off16 = ((kk >> 2) * C::BLK + (kk & 3) * 32) >> 4;
+            const uint32_t off16 = C::L::kstep(kk) >> 4;
             mma_ss(tmem + C::TM_S + k * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_s_full(k));
@@ -357,10 +357,11 @@ __global__ void __launch_bounds__(384, 1)
               if (!(ok = mbar_wait(bar_p_full(k), tk[k] & 1, abort_flag, kSiteFwdMmaP))) break;
               tc_fence_after();
               const uint32_t tP = tmem + C::TM_S + k * 128;
-              const uint64_t dv = sdesc_sw128(opaque_u32(vaddr), C::BLK);
+              const uint64_t dv = C::L::desc_mn(opaque_u32(vaddr), C::L::BLKB);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step = 8 TMEM columns of packed P
-                mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, dv + kk * (2048 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, dv + kk * (C::L::ROWSTEP16 >> 4), idPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
               mma_commit(bar_pv_done(k));
               ++tk[k];
               if (j + 1 < n_kv_of(k)) {

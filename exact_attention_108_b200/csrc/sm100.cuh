@@ -228,6 +228,50 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// The same for any swizzle: layout 2 = 128-byte swizzle (rows of 128 bytes), 4 =
+// 64-byte swizzle (rows of 64 bytes); SBO = the stride of 8-row groups.
+__device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+
+// How a 128-row tile of D bf16 columns sits in shared memory: as D / CW blocks of
+// CW columns, each 128 rows of CW * 2 bytes, swizzled the way the TMA writes them
+// (128-byte swizzle for 64-column blocks, 64-byte swizzle for 32-column blocks).
+// Head dims 64 and 128 use 64-column blocks, 32 and 96 use 32-column blocks, so
+// that no TMA box is wider than a row.
+template <int D>
+struct Cols {
+  static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim 32, 64, 96 or 128");
+  static constexpr int CW = (D % 64 == 0) ? 64 : 32;     // columns per block
+  static constexpr int NB = D / CW;                      // blocks per row
+  static constexpr int ROWB = CW * 2;                    // bytes per block row
+  static constexpr int BLKB = 128 * ROWB;                // bytes per 128-row block
+  static constexpr uint32_t LAYOUT = (CW == 64) ? 2u : 4u;
+  static constexpr uint32_t SBO = 8 * ROWB;              // 8-row groups
+  static constexpr int KSTEPS = CW / 16;                 // 16-element MMA K steps per block row
+  // K-major operand (rows = M or N, D along K): byte offset of K step kk
+  static __device__ __forceinline__ uint32_t kstep(int kk) {
+    return (uint32_t)((kk / KSTEPS) * BLKB + (kk % KSTEPS) * 32);
+  }
+  // MN-major operand with D along M/N and rows along K: bytes per 16-row K step
+  static constexpr uint32_t ROWSTEP16 = 16 * ROWB;
+  static __device__ __forceinline__ uint64_t desc_k(uint32_t saddr) { return sdesc_swz(saddr, 16, SBO, LAYOUT); }
+  static __device__ __forceinline__ uint64_t desc_mn(uint32_t saddr, uint32_t lbo) {
+    return sdesc_swz(saddr, lbo, SBO, LAYOUT);
+  }
+  // byte offset of 16-byte chunk `chunk` (0 .. ROWB/16 - 1) of `row` inside a block
+  static __device__ __forceinline__ uint32_t chunk_offset(uint32_t row, uint32_t chunk) {
+    return CW == 64 ? row * 128u + ((chunk ^ (row & 7u)) << 4) : row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+  }
+};
+
 // tcgen05.ld, 32 lanes x 32 bits, 32 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(

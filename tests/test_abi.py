@@ -56,7 +56,8 @@ def test_fwd_validation(lib):
     assert _fwd(lib, B=0) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, H=-1) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, N=0) == binding.FATTN_ERR_INVALID_ARG
-    assert _fwd(lib, d=96) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, d=80) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, d=16) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd(lib, B=1 << 14, H=1 << 10, N=1 << 8) == binding.FATTN_ERR_UNSUPPORTED  # 2^32 rows
     # 2^23 heads of 129 rows: under 2^31 rows, but 2^31 once each head is padded to whole tiles
@@ -72,16 +73,17 @@ def test_workspace_size(lib):
     def a256(x):
         return (x + 255) // 256 * 256
     # D and LSE*log2(e) per head padded to whole 128-row tiles, then the fp32 dQ accumulator
-    for (B, H, N, d) in [(1, 1, 128, 64), (4, 32, 4096, 128), (3, 5, 384, 128), (1, 1, 100, 64), (2, 3, 200, 128)]:
+    for (B, H, N, d) in [(1, 1, 128, 64), (4, 32, 4096, 128), (3, 5, 384, 128), (1, 1, 100, 64), (2, 3, 200, 128),
+                         (1, 2, 300, 32), (2, 1, 129, 96)]:
         padded = B * H * ((N + 127) // 128 * 128)
         assert lib.fattn_bwd_workspace_size(B, H, N, d) == 2 * a256(padded * 4) + a256(B * H * N * d * 4)
-    assert lib.fattn_bwd_workspace_size(1, 1, 128, 96) == 0
+    assert lib.fattn_bwd_workspace_size(1, 1, 128, 80) == 0
     assert lib.fattn_bwd_workspace_size(1, 1, 0, 64) == 0
 
 
 def _bwd(lib, ws=P, ws_bytes=None, d=64, N=128, **kw):
     if ws_bytes is None:
-        ws_bytes = lib.fattn_bwd_workspace_size(1, 1, N, d) if d in (64, 128) else 1 << 30
+        ws_bytes = lib.fattn_bwd_workspace_size(1, 1, N, d) if d in (32, 64, 96, 128) else 1 << 30
     args = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P)
     args.update(kw)
     return lib.fattn_bwd(args["q"], args["k"], args["v"], args["o"], args["do"], args["lse"], args["dq"],
@@ -92,7 +94,7 @@ def test_bwd_validation(lib):
     assert _bwd(lib, do=None) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, ws=None) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, ws_bytes=16) == binding.FATTN_ERR_INVALID_ARG
-    assert _bwd(lib, d=32) == binding.FATTN_ERR_UNSUPPORTED
+    assert _bwd(lib, d=48) == binding.FATTN_ERR_UNSUPPORTED
     assert _bwd(lib, N=200, ws_bytes=lib.fattn_bwd_workspace_size(1, 1, 200, 64) - 16) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, dq=P + 2) == binding.FATTN_ERR_ALIGNMENT
     assert _bwd(lib, ws=P + 16) == binding.FATTN_ERR_ALIGNMENT  # workspace wants 256 bytes
@@ -151,7 +153,7 @@ def test_fwd_ex_validation(lib):
     assert _fwd_ex(lib, dropout_p=1.0) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd_ex(lib, dropout_p=-0.1) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd_ex(lib, dropout_p=float("nan")) == binding.FATTN_ERR_INVALID_ARG
-    assert _fwd_ex(lib, d=96) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd_ex(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd_ex(lib, B=1 << 14, H=1 << 10, H_kv=1, N_q=128, N_k=128) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd_ex(lib, B=1 << 14, H=1 << 10, H_kv=1 << 10, N_q=1, N_k=128) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd_ex(lib, v=P + 8) == binding.FATTN_ERR_ALIGNMENT
@@ -201,5 +203,5 @@ def test_decode_validation(lib):
     assert _dec(lib, num_splits=-1) == binding.FATTN_ERR_INVALID_ARG
     assert _dec(lib, causal=3) == binding.FATTN_ERR_INVALID_ARG
     assert _dec(lib, scale=float("inf")) == binding.FATTN_ERR_INVALID_ARG
-    assert _dec(lib, d=32) == binding.FATTN_ERR_UNSUPPORTED
+    assert _dec(lib, d=48) == binding.FATTN_ERR_UNSUPPORTED
     assert _dec(lib, q=P + 4) == binding.FATTN_ERR_ALIGNMENT
