@@ -229,7 +229,84 @@ def gpu_smi_id(torch, dev):
 
 
 # ------------------------------------------------------------- GPU arm
-EXTRA_WORKLOADS = ("peaked_n8192", "long_n32768_causal", "fwd_d64", "fwd_d64_causal")
+EXTRA_WORKLOADS = ("train_d128_causal", "peaked_n8192", "long_n32768_causal", "fwd_d64", "fwd_d64_causal")
+
+
+DECODE_SHAPE = dict(B=8, H=32, H_kv=8, N_q=1, N_k=32768, d=128, causal=True)
+
+
+def time_deterministic_bwd(torch, binding, w, dev, stream, steps, warmup, peak, flush, seed_offset=0):
+    """The deterministic backward (dK/dV without dQ reduce-adds, then the separate dQ
+    pass), each call timed with CUDA events on the launching stream; L2 flushed before
+    every call (outside the timed region)."""
+    from exact_attention_108_b200.workloads import make_inputs
+
+    q, k, v, do = (t.to(dev) for t in make_inputs(w.B, w.H, w.N, w.d, w.seed + seed_offset, w.dist, True))
+    o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    p = binding.BwdParams(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), w.B, w.H, w.H, w.N, w.N, w.d,
+                          1 if w.causal else 0, w.scale, 0.0, 0, 0, 1, None, 0)
+    import ctypes
+    lib = binding.load()
+    ws = torch.empty(int(lib.fattn_bwd_ex_workspace_size(ctypes.byref(p))), device=dev, dtype=torch.uint8)
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    h = int(stream.cuda_stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(warmup + steps):
+        flush.zero_()
+        if i >= warmup:
+            evs[i - warmup][0].record(stream)
+        rc = lib.fattn_bwd_ex(ctypes.byref(p), h)
+        if rc != 0:
+            raise binding.FattnError(rc, "fattn_bwd_ex")
+        if i >= warmup:
+            evs[i - warmup][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    return {"bwd_ms": round(ms, 4), "bwd_tflops": round(w.bwd_flops() / ms / 1e9, 1),
+            "bwd_frac_of_peak": round(w.bwd_flops() / ms / 1e9 / peak, 4),
+            "path": "fattn_bwd_ex deterministic=1: preprocess, dK/dV without dQ, dQ pass"}
+
+
+def time_decode(torch, binding, dev, stream, steps, warmup, hbm_peak):
+    """Split-KV decoding: one new query row per sequence against a 32768-key cache,
+    B=8, H=32 query heads sharing H_kv=8 key/value heads, d=128, causal.  The cache
+    (1.07 GB) is far larger than L2, so every call streams it from HBM."""
+    c = DECODE_SHAPE
+    g = torch.Generator("cpu").manual_seed(5)
+    q = torch.randn((c["B"], c["H"], c["N_q"], c["d"]), generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn((c["B"], c["H_kv"], c["N_k"], c["d"]), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((c["B"], c["H_kv"], c["N_k"], c["d"]), generator=g).to(torch.bfloat16).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((c["B"], c["H"], c["N_q"]), device=dev, dtype=torch.float32)
+    ws = None
+    for _ in range(warmup):
+        binding.decode(q, k, v, causal=c["causal"], out=o, lse=lse, stream=stream)
+    import ctypes
+    p = binding.DecodeParams(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), c["B"], c["H"],
+                             c["H_kv"], c["N_q"], c["N_k"], c["N_k"], c["d"], 1, 1.0 / math.sqrt(c["d"]), 0, None, 0)
+    lib = binding.load()
+    need = int(lib.fattn_decode_workspace_size(ctypes.byref(p)))
+    ws = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    h = int(stream.cuda_stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream)
+        rc = lib.fattn_decode(ctypes.byref(p), h)
+        if rc != 0:
+            raise binding.FattnError(rc, "fattn_decode")
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    kv_bytes = 2 * c["B"] * c["H_kv"] * c["N_k"] * c["d"] * 2
+    qo_bytes = 2 * c["B"] * c["H"] * c["N_q"] * c["d"] * 2 + 4 * c["B"] * c["H"] * c["N_q"]
+    gbs = (kv_bytes + qo_bytes) / ms / 1e6
+    return {**c, "ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "peak_gbs": hbm_peak,
+            "frac": round(gbs / hbm_peak, 4), "bound": "hbm", "workspace_bytes": need,
+            "algorithmic_bytes": kv_bytes + qo_bytes,
+            "note": "K and V read once, Q read and O, LSE written; split-KV partials and the merge are not counted"}
 
 
 def time_other_workload(torch, binding, w, dev, stream, steps, warmup, peak, flush):
@@ -392,6 +469,12 @@ def run_fattn(args, rank, world, local_rank):
                 continue
             others[name] = time_other_workload(torch, binding, WORKLOADS[name], dev, stream,
                                                args.extra_steps, 3, peak, flush)
+        # the deterministic backward beside the default one on the d=128 workloads
+        for name in ("train_d128_causal", "peaked_n8192", "long_n32768_causal"):
+            det = time_deterministic_bwd(torch, binding, WORKLOADS[name], dev, stream, args.extra_steps, 3,
+                                         peak, flush)
+            others.setdefault(name, {})["deterministic_backward"] = det
+        others["decode"] = time_decode(torch, binding, dev, stream, args.extra_steps, 3, hbm)
         others["clocks"] = sampler2.stop()
         others["timing"] = ("median of per-step CUDA-event stage times; L2 flushed before every step "
                             "(outside the timed stages); fwd = fattn_fwd, bwd = fattn_bwd (3 kernels)")
@@ -420,6 +503,8 @@ def run_fattn(args, rank, world, local_rank):
                    "dist": w.dist, "global_batch": w.B * world,
                    "l2": "inputs larger than L2: each step reads Q, K, V, dO and O, "
                          f"{5 * w.B * w.H * w.N * w.d * 2 / 2**20:.0f} MiB in all (> 126 MB L2); no flush"},
+        "bwd_path": "fattn_bwd: dQ added by fp32 bulk reduce-adds (the faster of the two backwards here; "
+                    "the deterministic one is timed under other_workloads)",
         "fwd_tflops": round(fwd_tflops, 1), "bwd_tflops": round(bwd_tflops, 1),
         "fwd_frac_of_peak": round(fwd_tflops / peak, 4), "bwd_frac_of_peak": round(bwd_tflops / peak, 4),
         "stage_ms": {"fwd": round(fwd_ms, 4), "bwd_preprocess": round(pre_ms, 4),
