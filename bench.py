@@ -432,30 +432,62 @@ def run_fattn(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers (pinned)
     e2e = None
     if not args.no_e2e:
+        # Every step copies its inputs from pinned host memory and its gradients back.
+        # The copies run on their own streams with two device buffer sets, so the
+        # host-to-device copy of step i+1 and the device-to-host copy of step i-1
+        # overlap the compute of step i (as a training loop that prefetches would).
         pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
         outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (q_h, k_h, v_h)]
-        e_steps = max(1, min(args.steps, args.e2e_steps))
-        for rep in range(2):  # first pass warms the copy engines
-            barrier()
-            torch.cuda.synchronize(dev)
+        e_steps = max(2, min(args.steps, args.e2e_steps))
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_sets = [tuple(torch.empty_like(t) for t in (q, k, v, do)) for _ in range(2)]
+        out_sets = [tuple(torch.empty_like(t) for t in (q, k, v)) for _ in range(2)]
+        ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in_ready", "in_free", "out_ready", "out_free")}
+
+        def e2e_run(n):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(e_steps if rep else 1):
-                for dst, src in zip((q, k, v, do), pin):
-                    dst.copy_(src, non_blocking=True)
-                binding.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
-                binding.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+            e0.record(h2d_s)
+            for i in range(n):
+                sl = i % 2
+                with torch.cuda.stream(h2d_s):
+                    if i >= 2:
+                        h2d_s.wait_event(ev["in_free"][sl])
+                    for dst, src in zip(in_sets[sl], pin):
+                        dst.copy_(src, non_blocking=True)
+                    ev["in_ready"][sl].record(h2d_s)
+                stream.wait_event(ev["in_ready"][sl])
+                if i >= 2:
+                    stream.wait_event(ev["out_free"][sl])
+                qq, kk, vv, dd = in_sets[sl]
+                gq, gk, gv = out_sets[sl]
+                binding.fwd(qq, kk, vv, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+                binding.bwd(qq, kk, vv, o, lse, dd, causal=w.causal, scale=w.scale, dq=gq, dk=gk, dv=gv,
                             workspace=ws, stream=stream)
-                for dst, src in zip(outs, (dq, dk, dv)):
-                    dst.copy_(src, non_blocking=True)
-            e1.record(stream)
+                ev["in_free"][sl].record(stream)
+                ev["out_ready"][sl].record(stream)
+                with torch.cuda.stream(d2h_s):
+                    d2h_s.wait_event(ev["out_ready"][sl])
+                    for dst, src in zip(outs, out_sets[sl]):
+                        dst.copy_(src, non_blocking=True)
+                    ev["out_free"][sl].record(d2h_s)
+            e1.record(d2h_s)
             torch.cuda.synchronize(dev)
-        e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+            return e0.elapsed_time(e1)
+
+        barrier()
+        torch.cuda.synchronize(dev)
+        e2e_run(2)  # warms the copy engines
+        barrier()
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e2e_run(e_steps) / e_steps, world, dev)
+        del in_sets, out_sets
         e2e = {"value": whole_job_tflops(world, step_flops, e_ms), "unit": "TFLOPS",
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs),
                "ms_per_step": e_ms, "steps": e_steps,
-               "path": "pinned host Q,K,V,dO -> device; fattn_fwd; fattn_bwd; dQ,dK,dV -> pinned host"}
+               "path": "pinned host Q,K,V,dO -> device (copy stream); fattn_fwd; fattn_bwd; dQ,dK,dV -> pinned "
+                       "host (second copy stream); two device buffer sets, so copies overlap the neighbouring "
+                       "steps' compute; timed from the first copy's start to the last copy's end"}
 
     # ---- the other workloads of the throughput target, timed in the same run
     others = None

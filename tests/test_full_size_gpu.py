@@ -130,3 +130,65 @@ def test_zero_queries_closed_form_full_size(name):
     err = (o.double() - mean).abs()
     assert err.max().item() <= 1e-2 and err.mean().item() <= 1e-3
     assert (lse.double() - counts.log()).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("name", ["train_d128_causal", "peaked_n8192"])
+def test_deterministic_backward_full_size(name):
+    """The deterministic backward at full size: dK and dV are bit-equal to the default
+    backward's (the same products in the same order, without the dQ product); dQ
+    matches the oracle on sampled rows of every head and is the same on a second run."""
+    w = WORKLOADS[name]
+    cpu, (q, k, v, do) = gpu_inputs(w.B, w.H, w.N, w.d, w.seed, w.dist, with_do=True)
+    o, lse = binding.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    ref = binding.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale)
+    det = binding.bwd_ex(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, deterministic=True)
+    det2 = binding.bwd_ex(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, deterministic=True)
+    assert_device_ok()
+    assert torch.equal(det[1], ref[1]) and torch.equal(det[2], ref[2])
+    assert torch.equal(det[0], det2[0])
+    qc, kc, vc, doc = cpu
+    rng = np.random.default_rng(w.seed + 100)
+    worst = 0.0
+    for (b, h) in [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]:
+        rows = _sampled_rows(w.N, rng)
+        qh, kh, vh, doh = (to_f64(t[b, h]) for t in (qc, kc, vc, doc))
+        dq_r = oracle.ref_dq_rows(qh, kh, vh, doh, rows, w.causal, w.scale)
+        err = np.abs(to_f64(det[0][b, h, rows]) - dq_r).max()
+        worst = max(worst, err / np.abs(dq_r).max())
+        assert err <= 2e-2 * np.abs(dq_r).max(), f"dQ rows head ({b},{h}): {err:.3e}"
+    print(f"[parity] {name} deterministic dQ sampled rows: max-abs {worst:.2e} of the rows' max|ref|")
+
+
+def test_grouped_heads_dropout_training_shape():
+    """B=4, H=32 query heads over H_kv=8 key/value heads, N=4096, d=128, causal, dropout
+    0.1: O and LSE on sampled rows of every query head, dQ on sampled rows of labelled
+    heads, against the oracle's general form with the same Philox draws."""
+    B, H, H_kv, N, d, p, seed, offset = 4, 32, 8, 4096, 128, 0.1, 2024, 3
+    g = torch.Generator("cpu").manual_seed(12)
+    qc = torch.randn((B, H, N, d), generator=g).to(torch.bfloat16)
+    kc = torch.randn((B, H_kv, N, d), generator=g).to(torch.bfloat16)
+    vc = torch.randn((B, H_kv, N, d), generator=g).to(torch.bfloat16)
+    doc = torch.randn((B, H, N, d), generator=g).to(torch.bfloat16)
+    q, k, v, do = (t.cuda() for t in (qc, kc, vc, doc))
+    scale = 1.0 / np.sqrt(d)
+    o, lse = binding.fwd_ex(q, k, v, causal=True, scale=scale, dropout_p=p, seed=seed, offset=offset)
+    dq, dk, dv = binding.bwd_ex(q, k, v, o, lse, do, causal=True, scale=scale, dropout_p=p, seed=seed,
+                                offset=offset)
+    assert_device_ok()
+    pf = float(np.float32(p))
+    qd, kd, vd, dod = (to_f64(t) for t in (qc, kc, vc, doc))
+    rng = np.random.default_rng(13)
+    o_max = 0.0
+    for b in range(B):
+        for h in range(H):
+            rows = _sampled_rows(N, rng)
+            o_r, l_r = oracle.ref_fwd_general_rows(qd, kd, vd, b, h, rows, True, scale, pf, seed, offset)
+            err = np.abs(to_f64(o[b, h, rows]) - o_r)
+            o_max = max(o_max, float(err.max()))
+            assert err.max() <= 1e-2 / (1 - p), f"O rows head ({b},{h}): {err.max():.3e}"
+            check_lse(lse[b, h, rows], l_r, f"head ({b},{h}) rows", quiet=True)
+            if (b, h) in ((0, 0), (B - 1, H - 1)):
+                dq_r = oracle.ref_dq_general_rows(qd, kd, vd, dod, b, h, rows, True, scale, pf, seed, offset)
+                e = np.abs(to_f64(dq[b, h, rows]) - dq_r).max()
+                assert e <= 2e-2 * np.abs(dq_r).max(), f"dQ rows head ({b},{h}): {e:.3e}"
+    print(f"[parity] grouped heads + dropout, training shape: O sampled rows max-abs {o_max:.3e}")
