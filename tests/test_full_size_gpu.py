@@ -15,7 +15,7 @@ import torch
 import oracle
 from exact_attention_108_b200 import binding
 from exact_attention_108_b200.workloads import WORKLOADS, to_f64
-from gpu_common import assert_device_ok, check_grad, check_lse, check_o, gpu_inputs
+from gpu_common import assert_device_ok, check_grad, check_lse, check_o, gpu_inputs, o_max_abs_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -185,7 +185,10 @@ def test_grouped_heads_dropout_training_shape():
             o_r, l_r = oracle.ref_fwd_general_rows(qd, kd, vd, b, h, rows, True, scale, pf, seed, offset)
             err = np.abs(to_f64(o[b, h, rows]) - o_r)
             o_max = max(o_max, float(err.max()))
-            assert err.max() <= 1e-2 / (1 - p), f"O rows head ({b},{h}): {err.max():.3e}"
+            # the dropout bound (reading 15) plus the bf16 rounding of O where |O| >= 2:
+            # the first causal rows average few, rescaled values and reach |O| of 2 to 8
+            excess = err - o_max_abs_bound(o_r, 1e-2 / (1 - p))
+            assert excess.max() <= 0, f"O rows head ({b},{h}): {err.max():.3e} (over by {excess.max():.3e})"
             check_lse(lse[b, h, rows], l_r, f"head ({b},{h}) rows", quiet=True)
             if (b, h) in ((0, 0), (B - 1, H - 1)):
                 dq_r = oracle.ref_dq_general_rows(qd, kd, vd, dod, b, h, rows, True, scale, pf, seed, offset)

@@ -11,7 +11,7 @@ import torch
 import oracle
 from exact_attention_108_b200 import binding
 from exact_attention_108_b200.workloads import to_f64
-from gpu_common import assert_device_ok, check_grad, check_o
+from gpu_common import assert_device_ok, check_grad, check_o, o_max_abs_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -77,9 +77,11 @@ def test_dropout_matches_oracle(B, H, H_kv, N_q, N_k, d, p, causal):
     qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
     pf = float(np.float32(p))  # the library takes dropout_p as fp32
     o_ref, lse_ref = oracle.ref_fwd_general(qf, kf, vf, causal, scale, pf, seed, offset)
-    # dropped weights are up to 1/(1-p) times larger, and so is the bf16 rounding of P
+    # dropped weights are up to 1/(1-p) times larger, and so is the bf16 rounding of P;
+    # the bf16 rounding of O itself comes on top where |O| >= 2
     err = np.abs(to_f64(o) - o_ref)
-    assert err.max() <= 1e-2 / (1 - p) and err.mean() <= 1e-3 / (1 - p), (err.max(), err.mean())
+    assert (err <= o_max_abs_bound(o_ref, 1e-2 / (1 - p))).all() and err.mean() <= 1e-3 / (1 - p), \
+        (err.max(), err.mean())
     _check_lse_general(lse, lse_ref)
     refs = oracle.ref_bwd_general(qf, kf, vf, dof, causal, scale, pf, seed, offset)
     for det, gs in grads.items():
