@@ -49,7 +49,7 @@ template <int D>
 struct DecodeCfg {
   using L = sm100::Cols<D>;
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int NSLOT = D == 128 ? 6 : D == 96 ? 8 : D == 64 ? 12 : 16;
+  static constexpr int NSLOT = D == 256 ? 2 : D == 128 ? 6 : D == 96 ? 8 : D == 64 ? 12 : 16;
   static constexpr int OFF_Q = 0, OFF_SLOT = TILE;
   static constexpr int OFF_BAR = OFF_SLOT + NSLOT * TILE;
   // q_full, slot_full[NSLOT], slot_empty[NSLOT], s_full[2], p_full[2], pv_done, o_done, drain
@@ -107,8 +107,18 @@ __global__ void __launch_bounds__(192, 1)
   const int hb = (int)((blockIdx.x / (unsigned)args.row_tiles) % (unsigned)args.kv_heads);
   const int split = (int)(blockIdx.x / ((unsigned)args.row_tiles * (unsigned)args.kv_heads));
   const int j0 = split * args.tiles_per_split;
-  const int j1 = min(args.num_kv_tiles, j0 + args.tiles_per_split);
-  const int n_kv = j1 - j0;  // >= 1: the host makes no empty split
+  int j1 = min(args.num_kv_tiles, j0 + args.tiles_per_split);
+  if (CAUSAL) {
+    // only the key tiles some row of this tile sees: up to key max_i + off, max_i the
+    // largest query index among the tile's packed rows (g * N_q + i)
+    const int p_first = rt * 128, p_last = min(args.rows, p_first + 128) - 1;
+    const int max_i = p_first / args.N_q != p_last / args.N_q ? args.N_q - 1 : p_last % args.N_q;
+    const int key_end = min(args.N_k, max_i + args.causal_off + 1);
+    j1 = min(j1, key_end <= 0 ? 0 : (key_end + 127) / 128);
+  }
+  // >= 1: a range whose rows see no key still runs one fully masked tile, so that its
+  // O = 0 and LSE = -inf are written
+  const int n_kv = max(1, j1 - j0);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
@@ -322,43 +332,44 @@ __global__ void __launch_bounds__(192, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, 0, abort_flag, kSiteDecSoftO));
     if (ok && warp_live) {
       tc_fence_after();
-      uint32_t o[D / 32][32];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld_wait(o[c]);
-      if (prow < args.rows) {
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no visible key in this range: 0
-        const float lse2 = m_ref + __log2f(l);         // -inf for such a row
+      const bool row_ok = prow < args.rows;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no visible key in this range: 0
+      const float lse2 = m_ref + __log2f(l);         // -inf for such a row
+      // O row, 32 columns at a time (a d = 256 row would not fit in registers at once):
+      // bf16 to O with one split, else fp32 to this split's partial
+      const size_t row = (size_t)hb * args.rows + prow;  // packed row (g, i) of key/value head hb
+      const size_t prow_all = ((size_t)split * args.kv_heads + hb) * args.rows + prow;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_ld_wait(o);
+        if (!row_ok) continue;
         if (args.splits == 1) {
-          // packed row (g, i) of key/value head hb is row hb * rows + prow of O and LSE
-          const size_t row = (size_t)hb * args.rows + prow;
-          uint4* dst = reinterpret_cast<uint4*>(args.o + row * D);
+          uint4* dst = reinterpret_cast<uint4*>(args.o + row * D + c * 32);
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c)
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint32_t* x = &o[c][q4 * 8];
-              dst[c * 4 + q4] = make_uint4(
-                  pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
-                  pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
-                  pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
-                  pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
-            }
-          args.lse[row] = lse2 * 0.69314718055994530942f;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t* x = &o[q4 * 8];
+            dst[q4] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
+          }
         } else {
-          const size_t prow_all = ((size_t)split * args.kv_heads + hb) * args.rows + prow;
-          float4* dst = reinterpret_cast<float4*>(args.o_part + prow_all * D);
+          float4* dst = reinterpret_cast<float4*>(args.o_part + prow_all * D + c * 32);
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c)
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const uint32_t* x = &o[c][q4 * 4];
-              dst[c * 8 + q4] = make_float4(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l,
-                                            __uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l);
-            }
-          args.lse_part[prow_all] = lse2;
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const uint32_t* x = &o[q4 * 4];
+            dst[q4] = make_float4(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l,
+                                  __uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l);
+          }
         }
+      }
+      if (row_ok) {
+        if (args.splits == 1)
+          args.lse[row] = lse2 * 0.69314718055994530942f;
+        else
+          args.lse_part[prow_all] = lse2;
       }
     }
     tc_fence_before();
@@ -385,7 +396,7 @@ __global__ void __launch_bounds__(256) fattn_decode_merge_kernel(const DecodeArg
   const size_t base = (size_t)hb * args.rows + prow;
   float m = -INFINITY;
   for (int s = 0; s < args.splits; ++s) m = fmaxf(m, args.lse_part[base + s * stride]);
-  constexpr int PER = D / 32;  // columns per lane: 1 to 4
+  constexpr int PER = D / 32;  // columns per lane: 1 to 8
   float acc[PER] = {};
   float wsum = 0.f;
   if (m != -INFINITY) {

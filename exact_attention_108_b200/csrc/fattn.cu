@@ -117,7 +117,9 @@ int check_problem(const Problem& p) {
   if (!std::isfinite(p.scale)) return FATTN_ERR_INVALID_ARG;
   if (p.causal != 0 && p.causal != 1) return FATTN_ERR_INVALID_ARG;
   if (!(p.dropout_p >= 0.f && p.dropout_p < 1.f)) return FATTN_ERR_INVALID_ARG;  // NaN fails too
-  if (p.d != 32 && p.d != 64 && p.d != 96 && p.d != 128) return FATTN_ERR_UNSUPPORTED;
+  if (p.d != 32 && p.d != 64 && p.d != 96 && p.d != 128 && p.d != 256) return FATTN_ERR_UNSUPPORTED;
+  // d = 256: the forward only (one query tile per CTA, see run_fwd), without dropout
+  if (p.d == 256 && p.dropout_p > 0.f) return FATTN_ERR_UNSUPPORTED;
   // rows, and rows rounded up to whole tiles per head, are counted in int
   if (p.q_heads() * padded_n(p.N_q) >= (1ll << 31) || p.kv_heads() * padded_n(p.N_k) >= (1ll << 31))
     return FATTN_ERR_UNSUPPORTED;
@@ -297,8 +299,18 @@ int fwd_dispatch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   return drop ? launch_fwd<D, false, true>(mq, mk, mv, a, st) : launch_fwd<D, false, false>(mq, mk, mv, a, st);
 }
 
+int decode_impl(const fattn_decode_params* x, cudaStream_t st);
+
 // The forward of a validated problem (pointers checked by the caller).
 int run_fwd(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse, cudaStream_t st) {
+  if (p.d == 256) {
+    // Two query tiles with their 256-column O accumulators do not fit in the 512 TMEM
+    // columns, so d = 256 runs the one-tile-per-CTA kernel of the decoding path with
+    // a single key split (it writes O and LSE itself and needs no workspace).
+    fattn_decode_params x{q, k, v, o, lse, p.B, p.H, p.H_kv, p.N_q, p.N_k, p.N_k, p.d, p.causal, p.scale, 1,
+                          nullptr, 0};
+    return decode_impl(&x, st);
+  }
   CUtensorMap mq, mk, mv;
   if (int rc = make_head_map(&mq, q, p.q_heads(), p.N_q, p.d)) return rc;
   if (int rc = make_head_map(&mk, k, p.kv_heads(), p.N_k, p.d)) return rc;
@@ -507,6 +519,13 @@ int launch_dq(void* dq, long long rows, float scale, const WsParts& w, cudaStrea
   return FATTN_OK;
 }
 
+// The backward's shape check: the forward's, without d = 256 (its tiles do not fit the
+// backward's shared memory and TMEM).
+int check_bwd_problem(const Problem& p) {
+  if (int rc = check_problem(p)) return rc;
+  return p.d == 256 ? FATTN_ERR_UNSUPPORTED : FATTN_OK;
+}
+
 int check_workspace(void* workspace, size_t bytes, const Problem& p, bool deterministic) {
   if (!workspace) return FATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FATTN_ERR_ALIGNMENT;
@@ -554,7 +573,7 @@ int check_decode(const fattn_decode_params& x) {
   if (x.B < 1 || x.H < 1 || x.H_kv < 1 || x.N_q < 1 || x.N_k < 1) return FATTN_ERR_INVALID_ARG;
   if (x.H % x.H_kv != 0 || x.N_k_cap < x.N_k) return FATTN_ERR_INVALID_ARG;
   if (!std::isfinite(x.scale) || (x.causal != 0 && x.causal != 1) || x.num_splits < 0) return FATTN_ERR_INVALID_ARG;
-  if (x.d != 32 && x.d != 64 && x.d != 96 && x.d != 128) return FATTN_ERR_UNSUPPORTED;
+  if (x.d != 32 && x.d != 64 && x.d != 96 && x.d != 128 && x.d != 256) return FATTN_ERR_UNSUPPORTED;
   const long long rows = (long long)(x.H / x.H_kv) * x.N_q;
   if ((long long)x.B * x.H_kv * ((rows + 127) / 128 * 128) >= (1ll << 31) ||
       (long long)x.B * x.H_kv * padded_n(x.N_k_cap) >= (1ll << 31))
@@ -650,14 +669,14 @@ int fattn_fwd_ex(const fattn_fwd_params* x, fattn_stream_t stream) {
 
 size_t fattn_bwd_workspace_size(int B, int H, int N, int d) {
   const Problem p = square(B, H, N, d, 0, 1.f);
-  if (check_problem(p) != FATTN_OK) return 0;
+  if (check_bwd_problem(p) != FATTN_OK) return 0;
   return ws_bytes_needed(p, false);
 }
 
 size_t fattn_bwd_ex_workspace_size(const fattn_bwd_params* x) {
   if (!x) return 0;
   const Problem p = problem_of(*x);
-  if (check_problem(p) != FATTN_OK) return 0;
+  if (check_bwd_problem(p) != FATTN_OK) return 0;
   return ws_bytes_needed(p, x->deterministic != 0);
 }
 
@@ -665,7 +684,7 @@ int fattn_bwd_preprocess(const void* o, const void* dout, const float* lse, int 
                          void* workspace, size_t workspace_bytes, fattn_stream_t stream) {
   if (!o || !dout || !lse || !workspace) return FATTN_ERR_INVALID_ARG;
   const Problem p = square(B, H, N, d, 0, 1.f);
-  if (int rc = check_problem(p)) return rc;
+  if (int rc = check_bwd_problem(p)) return rc;
   if (!aligned16(o) || !aligned16(dout) || !aligned16(lse)) return FATTN_ERR_ALIGNMENT;
   if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
   const WsParts w = split_workspace(workspace, p, false);
@@ -678,7 +697,7 @@ int fattn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout
                    fattn_stream_t stream) {
   if (!q || !k || !v || !dout || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
   const Problem p = square(B, H, N, d, causal, scale);
-  if (int rc = check_problem(p)) return rc;
+  if (int rc = check_bwd_problem(p)) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv))
     return FATTN_ERR_ALIGNMENT;
   if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
@@ -690,7 +709,7 @@ int fattn_bwd_dq(void* dq, int B, int H, int N, int d, float scale, void* worksp
                  fattn_stream_t stream) {
   if (!dq || !workspace) return FATTN_ERR_INVALID_ARG;
   const Problem p = square(B, H, N, d, 0, scale);
-  if (int rc = check_problem(p)) return rc;
+  if (int rc = check_bwd_problem(p)) return rc;
   if (!aligned16(dq)) return FATTN_ERR_ALIGNMENT;
   if (int rc = check_workspace(workspace, workspace_bytes, p, false)) return rc;
   const long long rows = p.q_heads() * N;
@@ -704,7 +723,7 @@ int fattn_bwd(const void* q, const void* k, const void* v, const void* o, const 
               size_t workspace_bytes, fattn_stream_t stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FATTN_ERR_INVALID_ARG;
   const Problem p = square(B, H, N, d, causal, scale);
-  if (int rc = check_problem(p)) return rc;
+  if (int rc = check_bwd_problem(p)) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FATTN_ERR_ALIGNMENT;
@@ -718,7 +737,7 @@ int fattn_bwd_ex(const fattn_bwd_params* x, fattn_stream_t stream) {
     return FATTN_ERR_INVALID_ARG;
   if (x->deterministic != 0 && x->deterministic != 1) return FATTN_ERR_INVALID_ARG;
   const Problem p = problem_of(*x);
-  if (int rc = check_problem(p)) return rc;
+  if (int rc = check_bwd_problem(p)) return rc;
   if (!aligned16(x->q) || !aligned16(x->k) || !aligned16(x->v) || !aligned16(x->o) || !aligned16(x->dout) ||
       !aligned16(x->lse) || !aligned16(x->dq) || !aligned16(x->dk) || !aligned16(x->dv))
     return FATTN_ERR_ALIGNMENT;
@@ -740,6 +759,14 @@ int fattn_decode(const fattn_decode_params* x, fattn_stream_t stream) {
   if (int rc = check_decode(*x)) return rc;
   if (!aligned16(x->q) || !aligned16(x->k) || !aligned16(x->v) || !aligned16(x->o) || !aligned16(x->lse))
     return FATTN_ERR_ALIGNMENT;
+  return decode_impl(x, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+// fattn_decode after validation (also the d = 256 forward).
+int decode_impl(const fattn_decode_params* x, cudaStream_t st) {
   int sms = 0;
   if (int rc = sm_count(&sms)) return rc;
   const DecodePlan pl = decode_plan(*x, sms);
@@ -772,11 +799,15 @@ int fattn_decode(const fattn_decode_params* x, fattn_stream_t stream) {
   a.kv_heads = (int)kv_heads;
   a.causal_off = x->N_k - x->N_q;
   a.scale_log2 = x->scale * kLog2e;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (x->d == 256)
+    return x->causal ? launch_decode<256, true>(mq, mk, mv, a, st) : launch_decode<256, false>(mq, mk, mv, a, st);
   return by_d(x->d, [&](auto D) {
     return x->causal ? launch_decode<D.value, true>(mq, mk, mv, a, st) : launch_decode<D.value, false>(mq, mk, mv, a, st);
   });
 }
+}  // namespace
+
+extern "C" {
 
 // ---------------------------------------------------------------------------
 // fattn_bwd_noalloc: the backward's scratch lives in this fixed device array
@@ -813,7 +844,7 @@ int fattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o
                       void* dq, void* dk, void* dv, int B, int H, int N, int d, int causal, float scale,
                       fattn_stream_t stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FATTN_ERR_INVALID_ARG;
-  if (int rc = check_problem(square(B, H, N, d, causal, scale))) return rc;
+  if (int rc = check_bwd_problem(square(B, H, N, d, causal, scale))) return rc;
   if (fattn_bwd_workspace_size(B, H, N, d) > (size_t)FATTN_NOALLOC_SCRATCH_BYTES) return FATTN_ERR_SCRATCH_TOO_SMALL;
   void* scratch = nullptr;
   if (int rc = noalloc_scratch(&scratch)) return rc;

@@ -244,11 +244,11 @@ __device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo_bytes
 // How a 128-row tile of D bf16 columns sits in shared memory: as D / CW blocks of
 // CW columns, each 128 rows of CW * 2 bytes, swizzled the way the TMA writes them
 // (128-byte swizzle for 64-column blocks, 64-byte swizzle for 32-column blocks).
-// Head dims 64 and 128 use 64-column blocks, 32 and 96 use 32-column blocks, so
-// that no TMA box is wider than a row.
+// Head dims 64, 128 and 256 use 64-column blocks, 32 and 96 use 32-column blocks,
+// so that no TMA box is wider than a row.
 template <int D>
 struct Cols {
-  static_assert(D == 32 || D == 64 || D == 96 || D == 128, "head dim 32, 64, 96 or 128");
+  static_assert(D == 32 || D == 64 || D == 96 || D == 128 || D == 256, "head dim 32, 64, 96, 128 or 256");
   static constexpr int CW = (D % 64 == 0) ? 64 : 32;     // columns per block
   static constexpr int NB = D / CW;                      // blocks per row
   static constexpr int ROWB = CW * 2;                    // bytes per block row

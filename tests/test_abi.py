@@ -57,8 +57,8 @@ def test_fwd_validation(lib):
     assert _fwd(lib, H=-1) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, N=0) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd(lib, d=80) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, d=512) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd(lib, d=16) == binding.FATTN_ERR_UNSUPPORTED
-    assert _fwd(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd(lib, B=1 << 14, H=1 << 10, N=1 << 8) == binding.FATTN_ERR_UNSUPPORTED  # 2^32 rows
     # 2^23 heads of 129 rows: under 2^31 rows, but 2^31 once each head is padded to whole tiles
     assert _fwd(lib, B=1 << 13, H=1 << 10, N=129) == binding.FATTN_ERR_UNSUPPORTED
@@ -95,6 +95,8 @@ def test_bwd_validation(lib):
     assert _bwd(lib, ws=None) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, ws_bytes=16) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, d=48) == binding.FATTN_ERR_UNSUPPORTED
+    assert _bwd(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED  # d = 256: forward only
+    assert lib.fattn_bwd_workspace_size(1, 1, 128, 256) == 0
     assert _bwd(lib, N=200, ws_bytes=lib.fattn_bwd_workspace_size(1, 1, 200, 64) - 16) == binding.FATTN_ERR_INVALID_ARG
     assert _bwd(lib, dq=P + 2) == binding.FATTN_ERR_ALIGNMENT
     assert _bwd(lib, ws=P + 16) == binding.FATTN_ERR_ALIGNMENT  # workspace wants 256 bytes
@@ -153,7 +155,8 @@ def test_fwd_ex_validation(lib):
     assert _fwd_ex(lib, dropout_p=1.0) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd_ex(lib, dropout_p=-0.1) == binding.FATTN_ERR_INVALID_ARG
     assert _fwd_ex(lib, dropout_p=float("nan")) == binding.FATTN_ERR_INVALID_ARG
-    assert _fwd_ex(lib, d=256) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd_ex(lib, d=512) == binding.FATTN_ERR_UNSUPPORTED
+    assert _fwd_ex(lib, d=256, dropout_p=0.1) == binding.FATTN_ERR_UNSUPPORTED  # d = 256: no dropout
     assert _fwd_ex(lib, B=1 << 14, H=1 << 10, H_kv=1, N_q=128, N_k=128) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd_ex(lib, B=1 << 14, H=1 << 10, H_kv=1 << 10, N_q=1, N_k=128) == binding.FATTN_ERR_UNSUPPORTED
     assert _fwd_ex(lib, v=P + 8) == binding.FATTN_ERR_ALIGNMENT

@@ -4,6 +4,7 @@ a second shared-memory layout in every kernel.  Parity with the fp64 oracle for
 the forward, both backwards and decoding, on several tiles with ragged ends."""
 import math
 
+import numpy as np
 import pytest
 import torch
 
@@ -64,3 +65,43 @@ def test_head_dim_grouped_uneven_lengths(d):
     od_ref, ld_ref = oracle.ref_fwd_general(qf[:, :, -3:], kf, vf, True, scale)
     check_o(od, od_ref, f"d={d} decode")
     check_lse(ld, ld_ref, f"d={d} decode")
+
+
+D256_CASES = [
+    # B, H, H_kv, N_q, N_k, causal
+    (1, 2, 2, 384, 384, False),
+    (1, 2, 2, 384, 384, True),
+    (2, 4, 2, 300, 1000, True),    # grouped heads, N_q < N_k, ragged
+    (1, 2, 1, 500, 200, True),     # N_q > N_k: rows 0..299 see no key
+    (1, 3, 3, 1000, 1000, False),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,causal", D256_CASES)
+def test_head_dim_256_forward(B, H, H_kv, N_q, N_k, causal):
+    """d = 256: the forward runs the one-query-tile-per-CTA kernel of the decoding path
+    (two query tiles with their 256-column accumulators would not fit in TMEM)."""
+    d = 256
+    g = torch.Generator("cpu").manual_seed(80 + N_q)
+    q = torch.randn((B, H, N_q, d), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, H_kv, N_k, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, H_kv, N_k, d), generator=g).to(torch.bfloat16)
+    qg, kg, vg = (t.cuda() for t in (q, k, v))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=causal, scale=scale)
+    od, ld = binding.decode(qg[:, :, -4:].contiguous(), kg, vg, causal=causal, num_splits=3)
+    assert_device_ok()
+    qf, kf, vf = (to_f64(t) for t in (q, k, v))
+    o_ref, lse_ref = oracle.ref_fwd_general(qf, kf, vf, causal, scale)
+    check_o(o, o_ref, "d=256")
+    g_lse = lse.double().cpu().numpy()
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(g_lse), empty)
+    assert np.abs(g_lse[~empty] - lse_ref[~empty]).max() <= 1e-3
+    od_ref, ld_ref = oracle.ref_fwd_general(qf[:, :, -4:], kf, vf, causal, scale)
+    check_o(od, od_ref, "d=256 decode")
+    check_lse(ld, ld_ref, "d=256 decode")
+    if B * H == 2 and N_q == N_k:  # the plain entry point takes the same path
+        o2, l2 = binding.fwd(qg, kg, vg, causal=causal, scale=scale)
+        assert_device_ok()
+        assert torch.equal(o, o2) and torch.equal(lse, l2)
