@@ -624,7 +624,8 @@ const char* fattn_status_string(int status) {
     case FATTN_OK: return "ok";
     case FATTN_ERR_INVALID_ARG: return "invalid argument";
     case FATTN_ERR_UNSUPPORTED:
-      return "unsupported shape (need d in {32,64,96,128} and B*H*ceil(N_q/128)*128, B*H_kv*ceil(N_k/128)*128 < 2^31)";
+      return "unsupported shape (need d in {32,64,96,128}, or 256 for the forward and decoding without dropout, "
+             "and B*H*ceil(N_q/128)*128, B*H_kv*ceil(N_k/128)*128 < 2^31)";
     case FATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
     case FATTN_ERR_CUDA: return "CUDA error (see fattn_last_cuda_error)";
     case FATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out on the device";

@@ -26,7 +26,9 @@
  * All pointers are DEVICE pointers on the current CUDA device and must be
  * 16-byte aligned.  Outputs must not alias inputs.
  *
- * Supported shapes: B, H, N >= 1 (any N); d in {64, 128};
+ * Supported shapes: B, H, N >= 1 (any N); d in {32, 64, 96, 128} for the
+ * forward and both backwards, and d = 256 for the forward and decoding only
+ * (without dropout; the backward entry points return FATTN_ERR_UNSUPPORTED);
  * B * H * ceil(N / 128) * 128 < 2^31.  scale must be finite (any sign).  The
  * kernels work on 128-row tiles; a ragged last tile of each head is masked
  * (keys past N never receive weight, and rows past N are neither read nor
@@ -66,7 +68,7 @@ typedef struct CUstream_st* fattn_stream_t; /* same object as cudaStream_t */
 typedef enum {
   FATTN_OK = 0,
   FATTN_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, non-finite scale, too small workspace */
-  FATTN_ERR_UNSUPPORTED = 2,    /* d not in {64,128}, size overflow */
+  FATTN_ERR_UNSUPPORTED = 2,    /* head dim not supported by this call, size overflow */
   FATTN_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
   FATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed; see fattn_last_cuda_error() */
   FATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out */
