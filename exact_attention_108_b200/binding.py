@@ -28,7 +28,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20  # FATTN_NOALLOC_SCRATCH_BYTES
 EXPORTED = ("fattn_fwd", "fattn_bwd", "fattn_bwd_workspace_size", "fattn_bwd_preprocess",
             "fattn_bwd_dkdv", "fattn_bwd_dq", "fattn_status_string", "fattn_last_cuda_error",
             "fattn_device_status", "fattn_version", "fattn_bwd_noalloc", "fattn_fwd_ex",
-            "fattn_bwd_ex", "fattn_bwd_ex_workspace_size", "fattn_decode", "fattn_decode_workspace_size")
+            "fattn_bwd_ex", "fattn_bwd_ex_workspace_size", "fattn_decode", "fattn_decode_workspace_size", "fattn_selftest_wait_timeout")
 
 
 class FwdParams(ctypes.Structure):
@@ -114,6 +114,8 @@ def load():
     L.fattn_decode.restype = i
     L.fattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams)]
     L.fattn_decode_workspace_size.restype = sz
+    L.fattn_selftest_wait_timeout.argtypes = [vp]
+    L.fattn_selftest_wait_timeout.restype = i
     L.fattn_version.argtypes = []
     L.fattn_version.restype = i
     _lib = L
@@ -357,3 +359,12 @@ def decode(q, k_cache, v_cache, n_k: int | None = None, causal: bool = False, sc
     if rc != FATTN_OK:
         raise FattnError(rc, "fattn_decode")
     return out, lse
+
+
+def selftest_wait_timeout(stream=None):
+    """Enqueue the failure-detection self-test (fattn_selftest_wait_timeout): a kernel
+    whose bounded wait runs out after about a second; device_status() then reports
+    FATTN_ERR_DEVICE_TIMEOUT."""
+    rc = load().fattn_selftest_wait_timeout(_stream_handle(stream))
+    if rc != FATTN_OK:
+        raise FattnError(rc, "fattn_selftest_wait_timeout")

@@ -19,6 +19,25 @@
 #include "dq_kernel.cuh"
 #include "fwd_kernel.cuh"
 
+namespace fattn {
+constexpr int kSiteSelfTest = 0x7f1;
+
+// One warp waits on a barrier that expects one arrival which never comes; the
+// bounded wait gives up after sm100::kWaitLimitNs and records kSiteSelfTest.
+__global__ void __launch_bounds__(32) fattn_selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = sm100::smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncwarp();
+  (void)sm100::mbar_wait(b, 0, &abort_flag, kSiteSelfTest);
+}
+}  // namespace fattn
+
 namespace {
 
 thread_local std::string t_last_cuda_error;
@@ -647,6 +666,13 @@ int fattn_device_status(int clear) {
     if (e != cudaSuccess) return cuda_fail(e, "clear device status");
   }
   return v == 0 ? FATTN_OK : FATTN_ERR_DEVICE_TIMEOUT;
+}
+
+int fattn_selftest_wait_timeout(fattn_stream_t stream) {
+  fattn::fattn_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fattn_selftest_wait_kernel launch");
+  return FATTN_OK;
 }
 
 int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,

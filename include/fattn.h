@@ -293,6 +293,17 @@ const char* fattn_last_cuda_error(void);
  */
 int fattn_device_status(int clear);
 
+/*
+ * Failure-detection self-test: enqueues one small kernel whose single warp waits on
+ * an on-chip barrier that nothing completes, with the same bounded wait the
+ * attention kernels use.  After about one second the wait gives up, records its
+ * site in the device status word and the kernel returns; no fault, trap or hang is
+ * involved, and the context stays usable.  A following fattn_device_status()
+ * reports FATTN_ERR_DEVICE_TIMEOUT (and clears it if asked).  Lets a caller, or a
+ * test, check that timeouts are detected and reported on its device.
+ */
+int fattn_selftest_wait_timeout(fattn_stream_t stream);
+
 /* Library version, e.g. 0x000200 for 0.2.0. */
 int fattn_version(void);
 
