@@ -11,7 +11,7 @@ import torch
 import oracle
 from exact_attention_108_b200 import binding
 from exact_attention_108_b200.workloads import to_f64
-from gpu_common import assert_device_ok, check_grad, check_o, o_max_abs_bound
+from gpu_common import assert_device_ok, check_grad, check_o, gpu_inputs, o_max_abs_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -120,3 +120,60 @@ def test_square_general_call_equals_the_plain_entry_points():
     assert_device_ok()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])  # dK, dV: same kernel, fixed order
+
+
+@pytest.mark.parametrize("p", [0.1, 0.5])
+def test_dropout_tiny_workload(p):
+    """The tiny workload (B=1, H=1, N=128, d=64, non-causal, seed 0) with dropout:
+    forward and both backwards element by element against the oracle."""
+    from exact_attention_108_b200.workloads import WORKLOADS
+    w = WORKLOADS["tiny"]
+    (q, k, v, do), (qg, kg, vg, dog) = gpu_inputs(w.B, w.H, w.N, w.d, w.seed, w.dist)
+    seed, offset = 99, 5
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=w.causal, scale=w.scale, dropout_p=p, seed=seed, offset=offset)
+    grads = {det: binding.bwd_ex(qg, kg, vg, o, lse, dog, causal=w.causal, scale=w.scale, dropout_p=p, seed=seed,
+                                 offset=offset, deterministic=det) for det in (False, True)}
+    assert_device_ok()
+    pf = float(np.float32(p))
+    qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = oracle.ref_fwd_general(qf, kf, vf, w.causal, w.scale, pf, seed, offset)
+    err = np.abs(to_f64(o) - o_ref)
+    assert (err <= o_max_abs_bound(o_ref, 1e-2 / (1 - p))).all() and err.mean() <= 1e-3 / (1 - p)
+    _check_lse_general(lse, lse_ref)
+    refs = oracle.ref_bwd_general(qf, kf, vf, dof, w.causal, w.scale, pf, seed, offset)
+    for det, gs in grads.items():
+        for g, r, n in zip(gs, refs, ("dQ", "dK", "dV")):
+            check_grad(g, r, n, f"tiny p={p}")
+
+
+@pytest.mark.parametrize("p", [0.1, 0.5])
+def test_dropout_training_shape_sampled_heads(p):
+    """The training shape (B=4, H=32, N=4096, d=128, causal, seed 2) with dropout: O and
+    LSE of sampled rows on every head, and whole labelled heads (fwd and bwd) against
+    the oracle with the same Philox draws."""
+    from exact_attention_108_b200.workloads import WORKLOADS
+    w = WORKLOADS["train_d128_causal"]
+    (q, k, v, do), (qg, kg, vg, dog) = gpu_inputs(w.B, w.H, w.N, w.d, w.seed, w.dist)
+    seed, offset = 31337, 1
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=True, scale=w.scale, dropout_p=p, seed=seed, offset=offset)
+    dq, dk, dv = binding.bwd_ex(qg, kg, vg, o, lse, dog, causal=True, scale=w.scale, dropout_p=p, seed=seed,
+                                offset=offset)
+    assert_device_ok()
+    pf = float(np.float32(p))
+    rng = np.random.default_rng(5)
+    qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
+    for b in range(w.B):
+        for h in range(w.H):
+            rows = sorted({0, 1, 127, 128, w.N - 1} | set(rng.integers(0, w.N, 4).tolist()))
+            o_r, l_r = oracle.ref_fwd_general_rows(qf, kf, vf, b, h, rows, True, w.scale, pf, seed, offset)
+            err = np.abs(to_f64(o[b, h, rows]) - o_r)
+            assert (err <= o_max_abs_bound(o_r, 1e-2 / (1 - p))).all(), (b, h, err.max())
+            assert np.abs(lse[b, h, rows].double().cpu().numpy() - l_r).max() <= 1e-3
+    for (b, h) in [(0, 0), (w.B - 1, w.H - 1)]:
+        # whole heads through ref_fwd_general_rows: a sliced [1, 1] call would renumber the
+        # flattened head index b*H + h that the dropout draws depend on
+        o_full, _ = oracle.ref_fwd_general_rows(qf, kf, vf, b, h, np.arange(w.N), True, w.scale, pf, seed, offset)
+        err = np.abs(to_f64(o[b, h]) - o_full)
+        assert (err <= o_max_abs_bound(o_full, 1e-2 / (1 - p))).all() and err.mean() <= 1e-3 / (1 - p)
+        dq_r = oracle.ref_dq_general_rows(qf, kf, vf, dof, b, h, np.arange(w.N), True, w.scale, pf, seed, offset)
+        check_grad(to_f64(dq[b, h]), dq_r, "dQ", f"train p={p} head ({b},{h})")
