@@ -177,3 +177,45 @@ def test_dropout_training_shape_sampled_heads(p):
         assert (err <= o_max_abs_bound(o_full, 1e-2 / (1 - p))).all() and err.mean() <= 1e-3 / (1 - p)
         dq_r = oracle.ref_dq_general_rows(qf, kf, vf, dof, b, h, np.arange(w.N), True, w.scale, pf, seed, offset)
         check_grad(to_f64(dq[b, h]), dq_r, "dQ", f"train p={p} head ({b},{h})")
+
+
+def test_graph_capture_of_the_general_forms_matches_eager_bitwise():
+    """The grouped-head forward with dropout, the deterministic backward and split-KV
+    decoding captured in one CUDA graph and replayed: every output bit-equal to the
+    eager calls (all buffers, workspaces included, allocated before the capture)."""
+    _, (qg, kg, vg, dog) = _inputs(2, 8, 2, 512, 700, 128, 11)
+    kw = dict(causal=True, dropout_p=0.2, seed=7, offset=2)
+    o_e, l_e = binding.fwd_ex(qg, kg, vg, **kw)
+    g_e = binding.bwd_ex(qg, kg, vg, o_e, l_e, dog, deterministic=True, **kw)
+    qd = qg[:, :, -2:].contiguous()
+    od_e, ld_e = binding.decode(qd, kg, vg, causal=True, num_splits=3)
+    assert_device_ok()
+    o, l = torch.empty_like(o_e), torch.empty_like(l_e)
+    dq, dk, dv = (torch.empty_like(t) for t in g_e)
+    od, ld = torch.empty_like(od_e), torch.empty_like(ld_e)
+    ws_b = torch.empty(64 << 20, device="cuda", dtype=torch.uint8)
+    ws_d = torch.empty(16 << 20, device="cuda", dtype=torch.uint8)
+
+    def step():
+        binding.fwd_ex(qg, kg, vg, out=o, lse=l, **kw)
+        binding.bwd_ex(qg, kg, vg, o, l, dog, deterministic=True, dq=dq, dk=dk, dv=dv, workspace=ws_b, **kw)
+        binding.decode(qd, kg, vg, causal=True, num_splits=3, out=od, lse=ld, workspace=ws_d)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up outside the capture
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(2):
+        for t in (o, l, dq, dk, dv, od, ld):
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_e) and torch.equal(l, l_e)
+        assert torch.equal(dq, g_e[0]) and torch.equal(dk, g_e[1]) and torch.equal(dv, g_e[2])
+        assert torch.equal(od, od_e) and torch.equal(ld, ld_e)
+    del graph
+    assert_device_ok()
