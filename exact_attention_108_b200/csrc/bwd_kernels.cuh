@@ -147,7 +147,8 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_DS + DS_BYTES;
   // kv_full, q_full[NS], q_empty[NS], s_full, dp_full, p_full, ds_full, dq_full, dq_free, done, drain,
   // staged (dQ partial written to shared memory)
-  static constexpr int NBAR = 1 + 2 * NS + 9;
+  // + staged1, qb_full[NS], qb_empty[NS]: the stage's dO half has barriers of its own
+  static constexpr int NBAR = 1 + 2 * NS + 10 + 2 * NS;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16;  // the dynamic shared window starts 1024-byte aligned
   static constexpr int TMEM_COLS = 512;
@@ -208,7 +209,14 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t bar_s_full = bar0 + 8u * (1 + 2 * C::NS);
   const uint32_t bar_dp_full = bar_s_full + 8, bar_p_full = bar_s_full + 16, bar_ds_full = bar_s_full + 24;
   const uint32_t bar_dq_full = bar_s_full + 32, bar_dq_free = bar_s_full + 40, bar_done = bar_s_full + 48;
-  const uint32_t bar_drain = bar_s_full + 56, bar_staged = bar_s_full + 64;
+  const uint32_t bar_drain = bar_s_full + 56, bar_staged = bar_s_full + 64, bar_staged1 = bar_s_full + 72;
+  // A Q/dO stage is two halves with their own full/empty barriers: Q and the
+  // statistics (bar_q_full/bar_q_empty), and dO (bar_qb_full/bar_qb_empty).  The dQ^T
+  // partial is staged with warpgroup 0's 64 queries over the Q half and warpgroup 1's
+  // over the dO half, and each half goes back to the producer as soon as its own
+  // bulk reduce has read it, so that Q_{i+2} (needed first, for S) loads early.
+  auto bar_qb_full = [&](int s) { return bar0 + 8u * (1 + 2 * C::NS + 10 + s); };
+  auto bar_qb_empty = [&](int s) { return bar0 + 8u * (1 + 2 * C::NS + 10 + C::NS + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -271,6 +279,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar_q_full(s), 1);
       mbar_init(bar_q_empty(s), 1);
+      mbar_init(bar_qb_full(s), 1);
+      mbar_init(bar_qb_empty(s), 1);
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
@@ -280,7 +290,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar_dq_free, 256);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
-    mbar_init(bar_staged, 256);
+    mbar_init(bar_staged, 128);
+    mbar_init(bar_staged1, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -312,25 +323,33 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_3d(sV + kb * C::L::BLKB, &tm_v, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
         }
         int it = 0;
+        int half_issued = 0;  // stage halves whose loads went out (2 per step)
         Step sx;
         for (; it < n_it; ++it, sx.next(n_head)) {
           const int s = it % C::NS;
           if (!mbar_wait(bar_q_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
           const int q_tile = i_begin + sx.qi, qh = bh * args.G + sx.g;
           const size_t stat_row = (size_t)qh * args.stat_stride + q_tile * 128;
-          mbar_arrive_expect_tx(bar_q_full(s), 2 * C::TILE + 1024);
+          mbar_arrive_expect_tx(bar_q_full(s), C::TILE + 1024);
 #pragma unroll
-          for (int kb = 0; kb < C::L::NB; ++kb) {
+          for (int kb = 0; kb < C::L::NB; ++kb)
             tma_load_3d(sQ(s) + kb * C::L::BLKB, &tm_q, bar_q_full(s), kb * C::L::CW, q_tile * 128, qh);
-            tma_load_3d(sDO(s) + kb * C::L::BLKB, &tm_do, bar_q_full(s), kb * C::L::CW, q_tile * 128, qh);
-          }
           bulk_load(sStat(s), args.lse2 + stat_row, 512, bar_q_full(s));
           bulk_load(sStat(s) + 512, args.dvec + stat_row, 512, bar_q_full(s));
+          ++half_issued;
+          if (!mbar_wait(bar_qb_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
+          mbar_arrive_expect_tx(bar_qb_full(s), C::TILE);
+#pragma unroll
+          for (int kb = 0; kb < C::L::NB; ++kb)
+            tma_load_3d(sDO(s) + kb * C::L::BLKB, &tm_do, bar_qb_full(s), kb * C::L::CW, q_tile * 128, qh);
+          ++half_issued;
         }
         if (it < n_it) {  // aborted: let the copies already issued land
           mbar_wait_ns(bar_kv_full, 0, 100000000ull);
-          for (int i = (it > C::NS ? it - C::NS : 0); i < it; ++i)
-            mbar_wait_ns(bar_q_full(i % C::NS), (i / C::NS) & 1, 100000000ull);
+          for (int i = (it > C::NS ? it - C::NS : 0); i <= it && i < n_it; ++i) {
+            if (2 * i < half_issued) mbar_wait_ns(bar_q_full(i % C::NS), (i / C::NS) & 1, 100000000ull);
+            if (2 * i + 1 < half_issued) mbar_wait_ns(bar_qb_full(i % C::NS), (i / C::NS) & 1, 100000000ull);
+          }
         }
       }
       __syncwarp();
@@ -365,6 +384,10 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           issue_kxq(tA, sK, sQ(0));  // S^T_0
           mma_commit(bar_s_full);
+          ok = mbar_wait(bar_qb_full(0), 0, abort_flag, kSiteBwdMmaQ);
+        }
+        if (ok) {
+          tc_fence_after();
           issue_kxq(tB, sV, sDO(0));  // dP^T_0
           mma_commit(bar_dp_full);
         }
@@ -401,6 +424,7 @@ __global__ void __launch_bounds__(384, 1)
             mma_commit(bar_dq_full);
           } else {
             mma_commit(bar_q_empty(s));  // dV_i and dK_i were the stage's last readers
+            mma_commit(bar_qb_empty(s));
           }
           if (it + 1 < n_it) {
             const int s1 = (it + 1) % C::NS;
@@ -414,8 +438,9 @@ __global__ void __launch_bounds__(384, 1)
             // product, once dP^T_i was read: the gradient warps did so before ds_full)
             if constexpr (WITH_DQ) {
               if (!(ok = mbar_wait(bar_dq_free, it & 1, abort_flag, kSiteBwdMmaDQ))) break;
-              tc_fence_after();
             }
+            if (!(ok = mbar_wait(bar_qb_full(s1), ((it + 1) / C::NS) & 1, abort_flag, kSiteBwdMmaQ))) break;
+            tc_fence_after();
             issue_kxq(tB, sV, sDO(s1));
             mma_commit(bar_dp_full);
           }
@@ -435,15 +460,24 @@ __global__ void __launch_bounds__(384, 1)
         Step sx;
         for (int it = 0; it < n_it; ++it, sx.next(n_head)) {
           const int s = it % C::NS;
-          if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
           // only the tile's rows inside the sequence (a ragged last tile has fewer)
           const int q_tile = i_begin + sx.qi;
           const int rows = q_tile == NT - 1 ? args.q_tail : 128;
+          const int rows0 = rows < 64 ? rows : 64, rows1 = rows - rows0;
           float* dst = args.dq_acc + ((size_t)(bh * args.G + sx.g) * args.N_q + q_tile * 128) * D;
-          bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows * D * 4));
+          // queries 0..63 (warpgroup 0), staged over the Q half; then 64..127 over the dO half
+          if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
+          bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows0 * D * 4));
           bulk_commit();
           bulk_wait_read0();
-          mbar_arrive(bar_q_empty(s));  // the producer may refill the stage
+          mbar_arrive(bar_q_empty(s));  // the producer may load the next Q here
+          if (!mbar_wait(bar_staged1, it & 1, abort_flag, kSiteBwdDrain)) break;
+          if (rows1 > 0) {
+            bulk_reduce_add_f32(dst + 64 * D, sDO(s), (uint32_t)(rows1 * D * 4));
+            bulk_commit();
+            bulk_wait_read0();
+          }
+          mbar_arrive(bar_qb_empty(s));  // ... and the next dO here
         }
         bulk_wait0();  // the last reduce has landed in global memory
       }
@@ -607,7 +641,7 @@ __global__ void __launch_bounds__(384, 1)
           st_shared_f32(sQ(s) + (uint32_t)((64 * h + c) * D + r) * 4u, __uint_as_float(v[c >> 5][c & 31]));
       }
       fence_async_shared();
-      mbar_arrive(bar_staged);
+      mbar_arrive(h == 0 ? bar_staged : bar_staged1);
     }
     if (h == 1) {
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort_flag, kSiteBwdEpi));
