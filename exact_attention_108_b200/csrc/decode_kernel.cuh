@@ -25,6 +25,8 @@
 // never stored.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fattn {
@@ -252,27 +254,33 @@ __global__ void __launch_bounds__(192, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(v[c]);
-        if (clip) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= lim) v[c >> 5][c & 31] = __float_as_uint(masked);
-        }
         float pm[4] = {masked, masked, masked, masked};
-        if (sl2 >= 0.f) {
+        auto mask_max = [&](auto clip_c) {
+          if constexpr (decltype(clip_c)::value) {
 #pragma unroll
-          for (int c = 0; c < 128; c += 8)
+            for (int c = 0; c < 128; ++c)
+              if (c >= lim) v[c >> 5][c & 31] = __float_as_uint(masked);
+          }
+          if (sl2 >= 0.f) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
-                            __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
-        } else {
+            for (int c = 0; c < 128; c += 8)
 #pragma unroll
-          for (int c = 0; c < 128; c += 8)
+              for (int u = 0; u < 4; ++u)
+                pm[u] = fmax3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                              __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+          } else {
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
-                            __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
-        }
+            for (int c = 0; c < 128; c += 8)
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                pm[u] = fmin3(pm[u], __uint_as_float(v[(c + 2 * u) >> 5][(c + 2 * u) & 31]),
+                              __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
+          }
+        };
+        if (clip)
+          mask_max(std::true_type{});
+        else
+          mask_max(std::false_type{});
         float mx = sl2 >= 0.f ? fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3])) : fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
         mx *= sl2;
         // the reference max moves only when a row max exceeds it by more than 2^8
@@ -301,27 +309,35 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[2][32];
+        // two copies of the unrolled loop, with and without the mask, picked once per
+        // tile (a test inside the loop would be paid for as selects on every tile)
+        auto exps = [&](auto clip_c) {
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
-                                             __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
-                                     sl2x2, negm2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = ex2(x0), p1 = ex2(x1);
-          if (clip) {  // a select, not the exponential, zeroes masked keys (-inf * 0 at scale 0)
-            p0 = c < lim ? p0 : 0.f;
-            p1 = c + 1 < lim ? p1 : 0.f;
+          for (int c = 0; c < 128; c += 2) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
+                                               __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
+                                       sl2x2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float p0 = ex2(x0), p1 = ex2(x1);
+            if constexpr (decltype(clip_c)::value) {  // a select, not the exponential, zeroes
+              p0 = c < lim ? p0 : 0.f;                // masked keys (-inf * 0 at scale 0)
+              p1 = c + 1 < lim ? p1 : 0.f;
+            }
+            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
+            pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
           }
-          acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
-          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
-        }
-        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-        float s0, s1;
-        f2_unpack(a2, s0, s1);
-        l += s0 + s1;
+          const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float s0, s1;
+          f2_unpack(a2, s0, s1);
+          l += s0 + s1;
+        };
+        if (clip)
+          exps(std::true_type{});
+        else
+          exps(std::false_type{});
         tmem_st32(tS, pk[0]);
         tmem_st32(tS + 32, pk[1]);
         tmem_st_wait();

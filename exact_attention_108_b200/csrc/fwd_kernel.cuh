@@ -38,6 +38,8 @@
 // and l share the same reference the final O / l is unchanged.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fattn {
@@ -428,18 +430,22 @@ __global__ void __launch_bounds__(384, 1)
         const int base = 128 * (q_tile - j) + args.causal_off + 1;
         const bool clip = CAUSAL ? base < 128 : (j == NKT - 1 && args.kv_tail < 128);
         const int lim = CAUSAL ? base + r : args.kv_tail;
+        // The mask is uniform over the tile, so the masked and the unmasked tiles
+        // get their own copies of the unrolled loops, picked by one branch per
+        // tile: a test inside the unrolled loops would be if-converted into compares
+        // and selects that every tile pays for.
         const float masked = sl2 >= 0.f ? -INFINITY : INFINITY;
         float mx;
+        tmem_ld32(tS, v[0]);
+        tmem_ld32(tS + 32, v[1]);
+        tmem_ld_wait(v[0]);
+        tmem_ld_wait(v[1]);
+        tmem_ld32(tS + 64, v[2]);
+        tmem_ld32(tS + 96, v[3]);
         {
-          tmem_ld32(tS, v[0]);
-          tmem_ld32(tS + 32, v[1]);
-          tmem_ld_wait(v[0]);
-          tmem_ld_wait(v[1]);
-          tmem_ld32(tS + 64, v[2]);
-          tmem_ld32(tS + 96, v[3]);
           float pm[4] = {masked, masked, masked, masked};
-          auto half = [&](int h) {
-            if (clip) {
+          auto half = [&](int h, auto clip_c) {
+            if constexpr (decltype(clip_c)::value) {
   #pragma unroll
               for (int c = h * 64; c < h * 64 + 64; ++c)
                 if (c >= lim) v[c >> 5][c & 31] = __float_as_uint(masked);
@@ -460,10 +466,17 @@ __global__ void __launch_bounds__(384, 1)
                                 __uint_as_float(v[(c + 2 * u + 1) >> 5][(c + 2 * u + 1) & 31]));
             }
           };
-          half(0);
-          tmem_ld_wait(v[2]);
-          tmem_ld_wait(v[3]);
-          half(1);
+          if (clip) {
+            half(0, std::true_type{});
+            tmem_ld_wait(v[2]);
+            tmem_ld_wait(v[3]);
+            half(1, std::true_type{});
+          } else {
+            half(0, std::false_type{});
+            tmem_ld_wait(v[2]);
+            tmem_ld_wait(v[3]);
+            half(1, std::false_type{});
+          }
           mx = sl2 >= 0.f ? fmax3(pm[0], pm[1], fmaxf(pm[2], pm[3])) : fmin3(pm[0], pm[1], fminf(pm[2], pm[3]));
           mx *= sl2;
         }
@@ -494,42 +507,55 @@ __global__ void __launch_bounds__(384, 1)
         // be trusted to give 0.
         // Dropout (page 2's op chain: softmax, dropout, then V): the undropped
         // weights go into the row sum l, the dropped and rescaled ones into P V.
-        uint32_t keep = 0xffffffffu;  // keep bits of the current 32 keys
+        // Without dropout the loop is instantiated with and without the mask, as
+        // above; with dropout, whose keep bits already make it the longer loop, one
+        // copy tests the mask per element (a second copy would spill).
         const uint32_t q_row = (uint32_t)(q_tile * 128 + r);
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
-        uint32_t pk[2][32];                          // P row as packed bf16 pairs
+        uint32_t pk[2][32];  // P row as packed bf16 pairs
+        auto exps = [&](auto mode_c) {
+          constexpr int MODE = decltype(mode_c)::value;  // 0: no mask, 1: mask, 2: mask if clip
+          uint32_t keep = 0xffffffffu;                    // keep bits of the current 32 keys
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};     // packed partial row sums
   #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
-                                             __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
-                                     sl2x2, negm2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = ex2(x0), p1 = ex2(x1);
-          if (clip) {
-            p0 = (c < lim) ? p0 : 0.f;
-            p1 = (c + 1 < lim) ? p1 : 0.f;
-          }
-          acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
-          if constexpr (DROPOUT) {
-            if ((c & 31) == 0) {
-              keep = 0;
-  #pragma unroll
-              for (int u = 0; u < 8; ++u)  // keys c .. c + 31, four per generator call
-                keep |= dropout_keep4(args.drop, (uint32_t)w.bh, q_row, (uint32_t)((j * 128 + c) / 4 + u)) << (4 * u);
+          for (int c = 0; c < 128; c += 2) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
+                                               __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
+                                       sl2x2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float p0 = ex2(x0), p1 = ex2(x1);
+            if (MODE == 1 || (MODE == 2 && clip)) {
+              p0 = (c < lim) ? p0 : 0.f;
+              p1 = (c + 1 < lim) ? p1 : 0.f;
             }
-            const float ks = args.drop.scale_keep;
-            p0 = ((keep >> (c & 31)) & 1u) ? p0 * ks : 0.f;
-            p1 = ((keep >> ((c + 1) & 31)) & 1u) ? p1 * ks : 0.f;
+            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], f2_pack(p0, p1));
+            if constexpr (DROPOUT) {
+              if ((c & 31) == 0) {
+                keep = 0;
+  #pragma unroll
+                for (int u = 0; u < 8; ++u)  // keys c .. c + 31, four per generator call
+                  keep |= dropout_keep4(args.drop, (uint32_t)w.bh, q_row, (uint32_t)((j * 128 + c) / 4 + u))
+                          << (4 * u);
+              }
+              const float ks = args.drop.scale_keep;
+              p0 = ((keep >> (c & 31)) & 1u) ? p0 * ks : 0.f;
+              p1 = ((keep >> ((c + 1) & 31)) & 1u) ? p1 * ks : 0.f;
+            }
+            pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
           }
-          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
-        }
-        {
           const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
           float s0, s1;
           f2_unpack(a2, s0, s1);
           l += s0 + s1;
+        };
+        if constexpr (DROPOUT) {
+          exps(std::integral_constant<int, 2>{});
+        } else {
+          if (clip)
+            exps(std::integral_constant<int, 1>{});
+          else
+            exps(std::integral_constant<int, 0>{});
         }
         // P (bf16 pairs) over the first 64 columns of S_k
         tmem_st32(tS, pk[0]);
