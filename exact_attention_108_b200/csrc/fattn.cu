@@ -211,11 +211,14 @@ void causal_groups(int BH, long long work, long long longest, long long head_byt
 }
 
 // Counters for the causal forward's dynamic unit claiming, kSchedSlots pairs per
-// device.  A slot goes to a launch only once the event recorded after the slot's
-// previous launch has completed -- that launch's last CTA has returned the
-// counters to 0 -- so no two kernels in flight share one.  A launch being
-// captured into a CUDA graph, or one that finds every slot busy, schedules its
-// units statically instead.
+// device.  A launch may use a slot once the launch that used it before has
+// finished -- its last CTA returns the counters to 0 -- so no two kernels in
+// flight share one.  A slot whose event (recorded after its previous launch) has
+// completed is free.  When every slot is busy, as when a host thread queues many
+// calls ahead of the GPU, the launch takes the least recently handed-out slot and
+// its stream first waits on that slot's event: on the same stream that wait costs
+// nothing, since stream order already puts the launch after the previous one.  A
+// launch being captured into a CUDA graph schedules its units statically.
 constexpr int kSchedSlots = 16;
 static __device__ unsigned int g_fwd_sched[kSchedSlots][2];
 
@@ -228,8 +231,10 @@ struct SchedPool {
 };
 SchedPool g_sched_pool[kMaxDevices];
 
-// Picks a free slot (pool locked by the caller); -1 if none is usable.
-int sched_slot(SchedPool& pool, cudaStream_t st) {
+// Picks a slot (pool locked by the caller); -1 if none is usable.  *wait is set
+// when the slot may still be in use and the stream must wait on its event.
+int sched_slot(SchedPool& pool, cudaStream_t st, bool* wait) {
+  *wait = false;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -262,7 +267,10 @@ int sched_slot(SchedPool& pool, cudaStream_t st) {
     // error, but leave any other pending error for the launch check to report
     if (q == cudaErrorNotReady && cudaPeekAtLastError() == cudaErrorNotReady) (void)cudaGetLastError();
   }
-  return -1;
+  const int s = pool.next;
+  pool.next = (s + 1) % kSchedSlots;
+  *wait = true;
+  return s;
 }
 
 template <int D, bool CAUSAL, bool DROP>
@@ -293,7 +301,12 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   int slot = -1;
   if (CAUSAL && ctas > 1) {
     lock.lock();
-    slot = sched_slot(pool, st);
+    bool wait = false;
+    slot = sched_slot(pool, st, &wait);
+    if (slot >= 0 && wait) {
+      const cudaError_t we = cudaStreamWaitEvent(st, pool.ev[slot], 0);
+      if (we != cudaSuccess) return cuda_fail(we, "cudaStreamWaitEvent");
+    }
     if (slot >= 0) args.sched = pool.base + 2 * slot;
   }
   kern<<<dim3((unsigned)ctas), 384, smem, st>>>(mq, mk, mv, args);
