@@ -1,8 +1,9 @@
 """The persistent forward's work distribution.
 
 One CTA per SM loops over units of two query tiles; causal launches claim units
-from a device counter (one of a small pool of counter slots), while launches
-under CUDA-graph capture, or with every slot busy, take units round-robin.
+from a device counter (one of a small pool of counter slots; with every slot
+busy a launch reuses the least recently handed-out one behind a stream wait on
+its event), while launches under CUDA-graph capture take units round-robin.
 Which CTA computes a unit does not change its arithmetic, so every schedule
 must give bit-identical O and LSE; the oracle pins one of them.
 """
@@ -86,4 +87,26 @@ def test_concurrent_streams_reuse_counter_slots_bitwise():
     assert_device_ok()
     for (i, o, lse, s) in outs:
         o.record_stream(s)
+        assert torch.equal(o, ref[i][0]) and torch.equal(lse, ref[i][1]), f"launch of input {i} differs"
+
+
+def test_launches_queued_ahead_of_the_gpu_bitwise():
+    """Forty causal launches on one stream queued behind a long sleep, so that the
+    host runs ahead and every counter slot is still busy when most of them are
+    issued: each must reuse a slot behind its event and match its sequential run."""
+    inputs = [gpu_inputs(2, 16, 768, 128, 70 + i, with_do=False)[1][:3] for i in range(5)]
+    ref = [binding.fwd(q, k, v, causal=True) for (q, k, v) in inputs]
+    torch.cuda.synchronize()
+    assert_device_ok()
+    outs = []
+    torch.cuda._sleep(200_000_000)  # about 0.1 s of GPU time ahead of the launches
+    for rep in range(8):
+        for i, (q, k, v) in enumerate(inputs):
+            o = torch.empty_like(q)
+            lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+            binding.fwd(q, k, v, causal=True, out=o, lse=lse)
+            outs.append((i, o, lse))
+    torch.cuda.synchronize()
+    assert_device_ok()
+    for (i, o, lse) in outs:
         assert torch.equal(o, ref[i][0]) and torch.equal(lse, ref[i][1]), f"launch of input {i} differs"
