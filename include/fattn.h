@@ -82,12 +82,15 @@ typedef enum {
  *   causal  : 0 = no mask, 1 = query i attends keys 0..i.
  *   scale   : multiplies QK^T (usually 1/sqrt(d)).
  * One CTA per SM loops over units of two 128-row query tiles.  A causal launch
- * lets its CTAs claim units from one of the static counter pairs.  It takes a
- * pair only when the event recorded after that pair's previous launch has
- * completed; that launch returned the pair to zero.  A launch during stream
- * capture, or one that finds every pair busy, assigns units round-robin.  The
- * schedule does not change the results: every unit is computed the same way,
- * whichever CTA takes it.
+ * lets its CTAs claim units from one of the static counter pairs; the launch
+ * that used the pair before has returned it to zero when it finished.  A pair
+ * whose event (recorded after its previous launch) has completed is taken as it
+ * is.  When every pair is busy, the launch takes the least recently handed-out
+ * pair and makes `stream` wait on that pair's event first: nothing, if the
+ * previous launch is earlier on the same stream, and otherwise an ordering
+ * after that launch on its own stream.  A launch during stream capture assigns
+ * units round-robin.  The schedule does not change the results: every unit is
+ * computed the same way, whichever CTA takes it.
  */
 int fattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
               int B, int H, int N, int d, int causal, float scale,
