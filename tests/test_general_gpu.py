@@ -42,6 +42,9 @@ CASES = [
     (1, 2, 1, 512, 128, 64),    # more queries than keys: causal rows 0..383 see nothing
     (1, 6, 3, 200, 200, 64),    # square, ragged, grouped
     (2, 2, 2, 77, 333, 128),    # causal offset not a multiple of the tile
+    (1, 16, 1, 384, 384, 128),  # sixteen query heads share one key/value head
+    (1, 4, 2, 130, 700, 32),    # d = 32: grouped, ragged, fewer queries than keys
+    (1, 6, 3, 700, 130, 96),    # d = 96: grouped, ragged, more queries than keys
 ]
 
 
@@ -66,7 +69,8 @@ def test_general_shapes_match_oracle(B, H, H_kv, N_q, N_k, d, causal):
 
 @pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
 @pytest.mark.parametrize("p", [0.1, 0.5])
-@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d", [(1, 2, 1, 256, 384, 64), (1, 2, 2, 200, 200, 128)])
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,d", [(1, 2, 1, 256, 384, 64), (1, 2, 2, 200, 200, 128),
+                                             (1, 4, 2, 200, 333, 32), (1, 4, 2, 333, 200, 96)])
 def test_dropout_matches_oracle(B, H, H_kv, N_q, N_k, d, p, causal):
     (q, k, v, do), (qg, kg, vg, dog) = _inputs(B, H, H_kv, N_q, N_k, d, 7)
     scale, seed, offset = 1.0 / math.sqrt(d), 0x1234_5678_9ABC, 17
@@ -219,3 +223,26 @@ def test_graph_capture_of_the_general_forms_matches_eager_bitwise():
         assert torch.equal(od, od_e) and torch.equal(ld, ld_e)
     del graph
     assert_device_ok()
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_negative_scale_grouped_dropout(causal):
+    """A negative scale flips which key a row favours (the row max becomes a min of
+    the raw scores); with grouped heads, a ragged bottom-right mask and dropout."""
+    (q, k, v, do), (qg, kg, vg, dog) = _inputs(1, 4, 2, 200, 300, 64, 21)
+    scale, p, seed, offset = -0.1, 0.2, 99, 5
+    o, lse = binding.fwd_ex(qg, kg, vg, causal=causal, scale=scale, dropout_p=p, seed=seed, offset=offset)
+    grads = {det: binding.bwd_ex(qg, kg, vg, o, lse, dog, causal=causal, scale=scale, dropout_p=p, seed=seed,
+                                 offset=offset, deterministic=det) for det in (False, True)}
+    assert_device_ok()
+    qf, kf, vf, dof = (to_f64(t) for t in (q, k, v, do))
+    pf = float(np.float32(p))
+    o_ref, lse_ref = oracle.ref_fwd_general(qf, kf, vf, causal, np.float32(scale).item(), pf, seed, offset)
+    err = np.abs(to_f64(o) - o_ref)
+    assert (err <= o_max_abs_bound(o_ref, 1e-2 / (1 - p))).all() and err.mean() <= 1e-3 / (1 - p), \
+        (err.max(), err.mean())
+    _check_lse_general(lse, lse_ref)
+    refs = oracle.ref_bwd_general(qf, kf, vf, dof, causal, np.float32(scale).item(), pf, seed, offset)
+    for det, gs in grads.items():
+        for g, r, n in zip(gs, refs, ("dQ", "dK", "dV")):
+            check_grad(g, r, n, "negative scale " + ("deterministic" if det else "reduce-add"))
