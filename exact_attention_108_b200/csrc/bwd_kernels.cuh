@@ -178,7 +178,7 @@ enum : int {
 //                P^T and dS^T, thread = head-dim lane for its half of dQ^T.  Warps
 //                4..7 also write dK and dV at the end.
 //   warp 8       TMA producer (K, V once; Q/dO tiles through an NS-deep ring)
-//   warp 9       tcgen05 issuer (one thread)
+//   warp 9       tcgen05 issuer (the whole warp, one elected lane per instruction)
 //   warp 10      dQ reducer (one thread): one bulk reduce-add per query tile
 //   warp 11      idle
 // Per query tile i the tensor cores run
@@ -355,7 +355,9 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // --------------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      // The whole warp runs this loop; one elected lane issues each tcgen05
+      // instruction (mma_*_warp).
+      {
         constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // K|V (K-major) x Q|dO (K-major)
         constexpr uint32_t id_kv = idesc_bf16_f32(128, D, false, true);    // P^T|dS^T (TMEM) x dO|Q (MN)
         constexpr uint32_t id_q = idesc_bf16_f32(128, 128, true, true);    // K^T (MN) x dS^T (MN)
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off16 = C::L::kstep(kk) >> 4;
-            mma_ss(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
+            mma_ss_warp(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
           }
         };
         bool ok = mbar_wait(bar_kv_full, 0, abort_flag, kSiteBwdMmaKV);
@@ -383,13 +385,13 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) {
           tc_fence_after();
           issue_kxq(tA, sK, sQ(0));  // S^T_0
-          mma_commit(bar_s_full);
+          mma_commit_warp(bar_s_full);
           ok = mbar_wait(bar_qb_full(0), 0, abort_flag, kSiteBwdMmaQ);
         }
         if (ok) {
           tc_fence_after();
           issue_kxq(tB, sV, sDO(0));  // dP^T_0
-          mma_commit(bar_dp_full);
+          mma_commit_warp(bar_dp_full);
         }
         for (int it = 0; it < n_it && ok; ++it) {
           const int s = it % C::NS;
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t db = C::L::desc_mn(opaque_u32(sDO(s)), C::L::BLKB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // queries 16kk..: P^T of half kk/4 at columns 64*(kk/4) + 8*(kk%4)
-              mma_ts(tmem + C::TM_DV, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4), id_kv,
+              mma_ts_warp(tmem + C::TM_DV, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4), id_kv,
                      (it > 0 || kk > 0) ? 1u : 0u);
           }
           // dK += dS^T Q  (A = dS^T from TMEM, two 64-query halves)
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t db = C::L::desc_mn(opaque_u32(sQ(s)), C::L::BLKB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // dS^T of half kk/4 at columns 64*(kk/4) + 32 + 8*(kk%4)
-              mma_ts(tmem + C::TM_DK, tA + (kk >> 2) * 64 + 32 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4),
+              mma_ts_warp(tmem + C::TM_DK, tA + (kk >> 2) * 64 + 32 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4),
                      id_kv,
                      (it > 0 || kk > 0) ? 1u : 0u);
           }
@@ -420,11 +422,11 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t da = C::L::desc_mn(opaque_u32(sK), kt_lbo), db = sdesc_sw128(opaque_u32(sDS), C::DS_BLK);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // 16 keys per step: 16 rows of K, 16 rows of dS^T
-              mma_ss(tB, da + kk * (C::L::ROWSTEP16 >> 4), db + kk * (2048 >> 4), id_q, kk > 0 ? 1u : 0u);
-            mma_commit(bar_dq_full);
+              mma_ss_warp(tB, da + kk * (C::L::ROWSTEP16 >> 4), db + kk * (2048 >> 4), id_q, kk > 0 ? 1u : 0u);
+            mma_commit_warp(bar_dq_full);
           } else {
-            mma_commit(bar_q_empty(s));  // dV_i and dK_i were the stage's last readers
-            mma_commit(bar_qb_empty(s));
+            mma_commit_warp(bar_q_empty(s));  // dV_i and dK_i were the stage's last readers
+            mma_commit_warp(bar_qb_empty(s));
           }
           if (it + 1 < n_it) {
             const int s1 = (it + 1) % C::NS;
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(384, 1)
             // S^T_{i+1} over region A: the dV/dK products reading P^T/dS^T were
             // issued before it, and tcgen05.mma of one thread executes in order
             issue_kxq(tA, sK, sQ(s1));
-            mma_commit(bar_s_full);
+            mma_commit_warp(bar_s_full);
             // dP^T_{i+1} over region B once dQ^T_i has been drained (without the dQ
             // product, once dP^T_i was read: the gradient warps did so before ds_full)
             if constexpr (WITH_DQ) {
@@ -442,11 +444,11 @@ __global__ void __launch_bounds__(384, 1)
             if (!(ok = mbar_wait(bar_qb_full(s1), ((it + 1) / C::NS) & 1, abort_flag, kSiteBwdMmaQ))) break;
             tc_fence_after();
             issue_kxq(tB, sV, sDO(s1));
-            mma_commit(bar_dp_full);
+            mma_commit_warp(bar_dp_full);
           }
         }
-        if (ok) mma_commit(bar_done);
-        mma_commit(bar_drain);
+        if (ok) mma_commit_warp(bar_done);
+        mma_commit_warp(bar_drain);
         mbar_wait_ns(bar_drain, 0, 100000000ull);
       }
       __syncwarp();

@@ -18,7 +18,8 @@
 // one split the CTA writes the final bf16 O and natural-log LSE itself.
 //
 // Roles (192 threads): warps 0..3 softmax (thread = packed row), warp 4 TMA
-// producer (Q once, K_j, V_j through an NSLOT-deep ring), warp 5 tcgen05 issuer.
+// producer (Q once, K_j, V_j through an NSLOT-deep ring), warp 5 tcgen05 issuer (the
+// whole warp, one elected lane per instruction).
 // S goes to two TMEM buffers (columns 0 and 128), so S_{j+1} runs while the
 // softmax works on S_j; O accumulates at column 256.  Warps whose 32 rows are all
 // padding skip the exponentials: their P rows only feed output rows that are
@@ -180,7 +181,9 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop; one elected lane issues each tcgen05
+    // instruction (mma_*_warp).
+    {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
       constexpr uint32_t idPV = idesc_bf16_f32(128, D, false, true);    // P (TMEM) x V (MN-major)
       auto slot_addr = [&](int i) { return sSlot0 + (i % C::NSLOT) * C::TILE; };
@@ -192,10 +195,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off16 = C::L::kstep(kk) >> 4;
-          mma_ss(tmem + C::TM_S + (j & 1) * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
+          mma_ss_warp(tmem + C::TM_S + (j & 1) * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s_full(j & 1));
-        mma_commit(bar_slot_empty((2 * j) % C::NSLOT));  // K_j has been read
+        mma_commit_warp(bar_s_full(j & 1));
+        mma_commit_warp(bar_slot_empty((2 * j) % C::NSLOT));  // K_j has been read
       };
       bool ok = mbar_wait(bar_q_full, 0, abort_flag, kSiteDecMmaQ);
       for (int j = 0; j < 2 && j < n_kv && ok; ++j) {
@@ -212,9 +215,9 @@ __global__ void __launch_bounds__(192, 1)
         const uint64_t dv = C::L::desc_mn(opaque_u32(slot_addr(2 * j + 1)), C::L::BLKB);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::TM_O, tP + kk * 8, dv + kk * (C::L::ROWSTEP16 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_pv_done);
-        mma_commit(bar_slot_empty((2 * j + 1) % C::NSLOT));
+          mma_ts_warp(tmem + C::TM_O, tP + kk * 8, dv + kk * (C::L::ROWSTEP16 >> 4), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_warp(bar_pv_done);
+        mma_commit_warp(bar_slot_empty((2 * j + 1) % C::NSLOT));
         // S_{j+2} over buffer j & 1: P_j V_j, issued just before, reads it first
         if (j + 2 < n_kv) {
           if (!(ok = wait_slot(2 * j + 4, kSiteDecMmaK))) break;
@@ -222,8 +225,8 @@ __global__ void __launch_bounds__(192, 1)
           issue_s(j + 2);
         }
       }
-      if (ok) mma_commit(bar_o_done);  // every P_j V_j is in O
-      mma_commit(bar_drain);
+      if (ok) mma_commit_warp(bar_o_done);  // every P_j V_j is in O
+      mma_commit_warp(bar_drain);
       mbar_wait_ns(bar_drain, 0, 100000000ull);
     }
     __syncwarp();

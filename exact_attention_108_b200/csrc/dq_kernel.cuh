@@ -18,7 +18,8 @@
 //               key tile; thread = query row of the tile.  Both write the dQ rows
 //               at the end, warpgroup h the 32-column chunks c with c % 2 == h.
 //   warp 8      TMA producer: Q_i, dO_i once; K_j, V_j through an NSLOT-deep ring
-//   warp 9      tcgen05 issuer (one thread); warps 10, 11 idle
+//   warp 9      tcgen05 issuer (the whole warp, one elected lane per instruction);
+//               warps 10, 11 idle
 // Tensor memory (512 columns): S in two buffers (columns 0 and 128; dS, bf16,
 // overlays the first 32 columns of each 64-key half), dP at 256, dQ at 384.
 // Issue order: S_0 dP_0 | S_1 dQ_0 dP_1 | S_2 dQ_1 dP_2 | ...: the exponentials of
@@ -202,7 +203,9 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // --------------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      // The whole warp runs this loop; one elected lane issues each tcgen05
+      // instruction (mma_*_warp).
+      {
         constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // Q|dO (K-major) x K|V (K-major)
         constexpr uint32_t id_dq = idesc_bf16_f32(128, D, false, true);    // dS (TMEM) x K (MN-major)
         auto slot_addr = [&](int i) { return sSlot0 + (i % C::NSLOT) * C::TILE; };
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off16 = C::L::kstep(kk) >> 4;
-            mma_ss(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
+            mma_ss_warp(dst, da + off16, db + off16, id_s, kk > 0 ? 1u : 0u);
           }
         };
         bool ok = mbar_wait(bar_q_full, 0, abort_flag, kSiteDqMmaQ);
@@ -223,13 +226,13 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) {
           tc_fence_after();
           issue_rows(tmem + C::TM_S, sQ, slot_addr(0));  // S_0
-          mma_commit(bar_s_full(0));
+          mma_commit_warp(bar_s_full(0));
           ok = wait_slot(1, kSiteDqMmaV);
         }
         if (ok) {
           tc_fence_after();
           issue_rows(tmem + C::TM_DP, sDO, slot_addr(1));  // dP_0
-          mma_commit(bar_dp_full);
+          mma_commit_warp(bar_dp_full);
         }
         for (int j = 0; j < n_kv && ok; ++j) {
           const int kslot = 2 * j, vslot = 2 * j + 1;
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!(ok = wait_slot(kslot + 2, kSiteDqMmaK))) break;
             tc_fence_after();
             issue_rows(tmem + C::TM_S + ((j + 1) & 1) * 128, sQ, slot_addr(kslot + 2));
-            mma_commit(bar_s_full((j + 1) & 1));
+            mma_commit_warp(bar_s_full((j + 1) & 1));
           }
           // dQ += dS_j K_j  (A = dS_j from TMEM, two 64-key halves; 8 steps of 16 keys)
           if (!(ok = mbar_wait(bar_ds_full, j & 1, abort_flag, kSiteDqMmaDS))) break;
@@ -249,21 +252,21 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t db = C::L::desc_mn(opaque_u32(slot_addr(kslot)), C::L::BLKB);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // keys 16kk..: dS of half kk/4 at columns 64*(kk/4) + 8*(kk%4)
-              mma_ts(tmem + C::TM_DQ, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4), id_dq,
+              mma_ts_warp(tmem + C::TM_DQ, tA + (kk >> 2) * 64 + (kk & 3) * 8, db + kk * (C::L::ROWSTEP16 >> 4), id_dq,
                      (j > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar_slot_empty(kslot % C::NSLOT));
-          mma_commit(bar_slot_empty(vslot % C::NSLOT));  // V_j's product dP_j was issued earlier
+          mma_commit_warp(bar_slot_empty(kslot % C::NSLOT));
+          mma_commit_warp(bar_slot_empty(vslot % C::NSLOT));  // V_j's product dP_j was issued earlier
           if (j + 1 < n_kv) {
             // dP_{j+1}: the gradient warps read dP_j before they signalled dS_j
             if (!(ok = wait_slot(vslot + 2, kSiteDqMmaV))) break;
             tc_fence_after();
             issue_rows(tmem + C::TM_DP, sDO, slot_addr(vslot + 2));
-            mma_commit(bar_dp_full);
+            mma_commit_warp(bar_dp_full);
           }
         }
-        if (ok) mma_commit(bar_done);
-        mma_commit(bar_drain);
+        if (ok) mma_commit_warp(bar_done);
+        mma_commit_warp(bar_drain);
         mbar_wait_ns(bar_drain, 0, 100000000ull);
       }
       __syncwarp();

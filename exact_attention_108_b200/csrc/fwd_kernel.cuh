@@ -14,7 +14,8 @@
 //   warps 4..7  softmax group 1, thread = row of query tile 1   (208 registers)
 //   warp 8      TMA producer: Q tiles through a 3-buffer ring, K_j, V_j through
 //               an NSLOT-deep ring; it also hands the work units to the others
-//   warp 9      tcgen05 issuer (one thread); warps 10, 11 idle   (88 registers)
+//   warp 9      tcgen05 issuer (the whole warp, one elected lane per instruction);
+//               warps 10, 11 idle                                 (88 registers)
 //                 S0 = Q0 K_j^T, S1 = Q1 K_j^T          (TMEM, fp32)
 //                 O0 += P0 V_j,  O1 += P1 V_j           (P read from TMEM)
 // While group 0 turns S0 into P0 the tensor cores compute S1 (and vice versa),
@@ -291,7 +292,9 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // ----------------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      // The whole warp runs this loop; one elected lane issues each tcgen05
+      // instruction (mma_*_warp), and lane 0 alone makes the plain arrivals.
+      {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
         constexpr uint32_t idPV = idesc_bf16_f32(128, D, false, true);    // P (TMEM) x V (MN-major)
         auto slot_of = [&](int i) { return i % C::NSLOT; };
@@ -306,9 +309,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off16 = C::L::kstep(kk) >> 4;
-            mma_ss(tmem + C::TM_S + k * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
+            mma_ss_warp(tmem + C::TM_S + k * 128, dq + off16, dk + off16, idS, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar_s_full(k));
+          mma_commit_warp(bar_s_full(k));
         };
         int it = 0;          // ring position of the current unit's K_0
         int qs = 0;          // Q ring position of the current unit's Q0
@@ -319,7 +322,8 @@ __global__ void __launch_bounds__(384, 1)
           const int e = nu % C::NUNIT;
           if (!(ok = mbar_wait(bar_unit_full(e), (nu / C::NUNIT) & 1, abort_flag, kSiteFwdUnit))) break;
           const int u = unit_ring[e];
-          mbar_arrive(bar_unit_empty(e));
+          if (lane == 0) mbar_arrive(bar_unit_empty(e));
+          __syncwarp();
           if (u < 0) break;
           const Unit w = unit_of(u);
           const int nq = w.n_kv1 > 0 ? 2 : 1;
@@ -334,10 +338,10 @@ __global__ void __launch_bounds__(384, 1)
             if (!(ok = mbar_wait(bar_q_full(qbuf(k)), ((qs + k) / C::QBUF) & 1, abort_flag, kSiteFwdMmaQ))) break;
             tc_fence_after();
             issue_s(k, qbuf(k), slot_of(it0));
-            if (n_kv_of(k) == 1) mma_commit(bar_q_empty(qbuf(k)));  // Q_k's only product
+            if (n_kv_of(k) == 1) mma_commit_warp(bar_q_empty(qbuf(k)));  // Q_k's only product
           }
           if (!ok) break;
-          mma_commit(bar_slot_empty(slot_of(it0)));
+          mma_commit_warp(bar_slot_empty(slot_of(it0)));
           // Issue order: S0_0 S1_0 | PV0_0 S0_1 | PV1_0 S1_1 | PV0_1 S0_2 | ...  While one
           // softmax group works on S_k, the tensor cores run the other group's P V and
           // its next S.  S_k(j+1) overwrites the columns PV_k(j) reads P_k(j) from.
@@ -362,25 +366,25 @@ __global__ void __launch_bounds__(384, 1)
               const uint64_t dv = C::L::desc_mn(opaque_u32(vaddr), C::L::BLKB);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step = 8 TMEM columns of packed P
-                mma_ts(tmem + C::TM_O + k * D, tP + kk * 8, dv + kk * (C::L::ROWSTEP16 >> 4), idPV,
+                mma_ts_warp(tmem + C::TM_O + k * D, tP + kk * 8, dv + kk * (C::L::ROWSTEP16 >> 4), idPV,
                        (j > 0 || kk > 0) ? 1u : 0u);
-              mma_commit(bar_pv_done(k));
+              mma_commit_warp(bar_pv_done(k));
               ++tk[k];
               if (j + 1 < n_kv_of(k)) {
                 issue_s(k, qbuf(k), slot_of(itK1));
-                if (j + 2 == n_kv_of(k)) mma_commit(bar_q_empty(qbuf(k)));  // Q_k's last product
+                if (j + 2 == n_kv_of(k)) mma_commit_warp(bar_q_empty(qbuf(k)));  // Q_k's last product
               }
             }
             if (!ok) break;
-            mma_commit(bar_slot_empty(slot_of(itV)));
-            if (more) mma_commit(bar_slot_empty(slot_of(itK1)));
+            mma_commit_warp(bar_slot_empty(slot_of(itV)));
+            if (more) mma_commit_warp(bar_slot_empty(slot_of(itK1)));
           }
           it = it0 + 2 * w.n_kv;
           qs += nq;
           for (int k = 0; k < nq; ++k) ++uk[k];
         }
         // Make sure nothing this thread issued is still running before TMEM is freed.
-        mma_commit(bar_drain);
+        mma_commit_warp(bar_drain);
         mbar_wait_ns(bar_drain, 0, 100000000ull);
       }
       __syncwarp();
