@@ -178,7 +178,7 @@ enum : int {
 //                P^T and dS^T, thread = head-dim lane for its half of dQ^T.  Warps
 //                4..7 also write dK and dV at the end.
 //   warp 8       TMA producer (K, V once; Q/dO tiles through an NS-deep ring)
-//   warp 9       tcgen05 issuer (the whole warp, one elected lane per instruction)
+//   warp 9       tcgen05 issuer (the whole warp; lane 0 issues each instruction)
 //   warp 10      dQ reducer (one thread): one bulk reduce-add per query tile
 //   warp 11      idle
 // Per query tile i the tensor cores run
@@ -355,8 +355,8 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // --------------------------------------------------------- MMA issuer
-      // The whole warp runs this loop; one elected lane issues each tcgen05
-      // instruction (mma_*_warp).
+      // The whole warp runs this loop; lane 0 issues each tcgen05 instruction
+      // (mma_*_warp).
       {
         constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // K|V (K-major) x Q|dO (K-major)
         constexpr uint32_t id_kv = idesc_bf16_f32(128, D, false, true);    // P^T|dS^T (TMEM) x dO|Q (MN)

@@ -19,7 +19,7 @@
 //
 // Roles (192 threads): warps 0..3 softmax (thread = packed row), warp 4 TMA
 // producer (Q once, K_j, V_j through an NSLOT-deep ring), warp 5 tcgen05 issuer (the
-// whole warp, one elected lane per instruction).
+// whole warp; lane 0 issues each instruction).
 // S goes to two TMEM buffers (columns 0 and 128), so S_{j+1} runs while the
 // softmax works on S_j; O accumulates at column 256.  Warps whose 32 rows are all
 // padding skip the exponentials: their P rows only feed output rows that are
@@ -181,8 +181,8 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
-    // The whole warp runs this loop; one elected lane issues each tcgen05
-    // instruction (mma_*_warp).
+    // The whole warp runs this loop; lane 0 issues each tcgen05 instruction
+    // (mma_*_warp).
     {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
       constexpr uint32_t idPV = idesc_bf16_f32(128, D, false, true);    // P (TMEM) x V (MN-major)

@@ -18,7 +18,7 @@
 //               key tile; thread = query row of the tile.  Both write the dQ rows
 //               at the end, warpgroup h the 32-column chunks c with c % 2 == h.
 //   warp 8      TMA producer: Q_i, dO_i once; K_j, V_j through an NSLOT-deep ring
-//   warp 9      tcgen05 issuer (the whole warp, one elected lane per instruction);
+//   warp 9      tcgen05 issuer (the whole warp; lane 0 issues each instruction);
 //               warps 10, 11 idle
 // Tensor memory (512 columns): S in two buffers (columns 0 and 128; dS, bf16,
 // overlays the first 32 columns of each 64-key half), dP at 256, dQ at 384.
@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // --------------------------------------------------------- MMA issuer
-      // The whole warp runs this loop; one elected lane issues each tcgen05
-      // instruction (mma_*_warp).
+      // The whole warp runs this loop; lane 0 issues each tcgen05 instruction
+      // (mma_*_warp).
       {
         constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);  // Q|dO (K-major) x K|V (K-major)
         constexpr uint32_t id_dq = idesc_bf16_f32(128, D, false, true);    // dS (TMEM) x K (MN-major)

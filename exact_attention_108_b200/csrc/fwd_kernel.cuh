@@ -14,7 +14,7 @@
 //   warps 4..7  softmax group 1, thread = row of query tile 1   (208 registers)
 //   warp 8      TMA producer: Q tiles through a 3-buffer ring, K_j, V_j through
 //               an NSLOT-deep ring; it also hands the work units to the others
-//   warp 9      tcgen05 issuer (the whole warp, one elected lane per instruction);
+//   warp 9      tcgen05 issuer (the whole warp; lane 0 issues each instruction);
 //               warps 10, 11 idle                                 (88 registers)
 //                 S0 = Q0 K_j^T, S1 = Q1 K_j^T          (TMEM, fp32)
 //                 O0 += P0 V_j,  O1 += P1 V_j           (P read from TMEM)
@@ -292,8 +292,8 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 9) {
       // ----------------------------------------------------------- MMA issuer
-      // The whole warp runs this loop; one elected lane issues each tcgen05
-      // instruction (mma_*_warp), and lane 0 alone makes the plain arrivals.
+      // The whole warp runs this loop; lane 0 issues each tcgen05 instruction
+      // (mma_*_warp) and makes the plain arrivals.
       {
         constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
         constexpr uint32_t idPV = idesc_bf16_f32(128, D, false, true);    // P (TMEM) x V (MN-major)
