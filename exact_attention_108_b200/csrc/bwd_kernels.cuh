@@ -179,7 +179,7 @@ enum : int {
 //                4..7 also write dK and dV at the end.
 //   warp 8       TMA producer (K, V once; Q/dO tiles through an NS-deep ring)
 //   warp 9       tcgen05 issuer (the whole warp; lane 0 issues each instruction)
-//   warp 10      dQ reducer (one thread): one bulk reduce-add per query tile
+//   warp 10      dQ reducer (lane 0 issues): one bulk reduce-add per half of a query tile
 //   warp 11      idle
 // Per query tile i the tensor cores run
 //   ... dV_i | dK_i dQ_i S_{i+1} | dP_{i+1} | dV_{i+1} | ...
@@ -311,17 +311,23 @@ __global__ void __launch_bounds__(384, 1)
     regs_decrease<88>();
     if (warp == 8) {
       // ---------------------------------------------------------- producer
-      if (lane == 0) {
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_do);
-        mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
+      // The whole warp runs the loop and its waits; lane 0 alone issues the copies
+      // and the barrier transactions (one()).  A lone lane running the loop competes
+      // for issue slots with the gradient warps beside it.
+      {
+        auto one = [&](auto f) { if (lane == 0) f(); __syncwarp(); };
+        one([&] {
+          prefetch_tensormap(&tm_q);
+          prefetch_tensormap(&tm_k);
+          prefetch_tensormap(&tm_v);
+          prefetch_tensormap(&tm_do);
+          mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
 #pragma unroll
-        for (int kb = 0; kb < C::L::NB; ++kb) {
-          tma_load_3d(sK + kb * C::L::BLKB, &tm_k, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
-          tma_load_3d(sV + kb * C::L::BLKB, &tm_v, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
-        }
+          for (int kb = 0; kb < C::L::NB; ++kb) {
+            tma_load_3d(sK + kb * C::L::BLKB, &tm_k, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
+            tma_load_3d(sV + kb * C::L::BLKB, &tm_v, bar_kv_full, kb * C::L::CW, kv_tile * 128, bh);
+          }
+        });
         int it = 0;
         int half_issued = 0;  // stage halves whose loads went out (2 per step)
         Step sx;
@@ -330,18 +336,22 @@ __global__ void __launch_bounds__(384, 1)
           if (!mbar_wait(bar_q_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
           const int q_tile = i_begin + sx.qi, qh = bh * args.G + sx.g;
           const size_t stat_row = (size_t)qh * args.stat_stride + q_tile * 128;
-          mbar_arrive_expect_tx(bar_q_full(s), C::TILE + 1024);
+          one([&] {
+            mbar_arrive_expect_tx(bar_q_full(s), C::TILE + 1024);
 #pragma unroll
-          for (int kb = 0; kb < C::L::NB; ++kb)
-            tma_load_3d(sQ(s) + kb * C::L::BLKB, &tm_q, bar_q_full(s), kb * C::L::CW, q_tile * 128, qh);
-          bulk_load(sStat(s), args.lse2 + stat_row, 512, bar_q_full(s));
-          bulk_load(sStat(s) + 512, args.dvec + stat_row, 512, bar_q_full(s));
+            for (int kb = 0; kb < C::L::NB; ++kb)
+              tma_load_3d(sQ(s) + kb * C::L::BLKB, &tm_q, bar_q_full(s), kb * C::L::CW, q_tile * 128, qh);
+            bulk_load(sStat(s), args.lse2 + stat_row, 512, bar_q_full(s));
+            bulk_load(sStat(s) + 512, args.dvec + stat_row, 512, bar_q_full(s));
+          });
           ++half_issued;
           if (!mbar_wait(bar_qb_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, kSiteBwdProducer)) break;
-          mbar_arrive_expect_tx(bar_qb_full(s), C::TILE);
+          one([&] {
+            mbar_arrive_expect_tx(bar_qb_full(s), C::TILE);
 #pragma unroll
-          for (int kb = 0; kb < C::L::NB; ++kb)
-            tma_load_3d(sDO(s) + kb * C::L::BLKB, &tm_do, bar_qb_full(s), kb * C::L::CW, q_tile * 128, qh);
+            for (int kb = 0; kb < C::L::NB; ++kb)
+              tma_load_3d(sDO(s) + kb * C::L::BLKB, &tm_do, bar_qb_full(s), kb * C::L::CW, q_tile * 128, qh);
+          });
           ++half_issued;
         }
         if (it < n_it) {  // aborted: let the copies already issued land
@@ -458,7 +468,9 @@ __global__ void __launch_bounds__(384, 1)
       // i's Q/dO stage; one TMA bulk reduce-add puts it into the accumulator rows,
       // which are contiguous.  The stage goes back to the producer once the reduce
       // has read it, without holding up a gradient warp meanwhile.
-      if (WITH_DQ && lane == 0) {
+      // As in the producer, the whole warp runs the loop, lane 0 issues (one()).
+      if (WITH_DQ) {
+        auto one = [&](auto f) { if (lane == 0) f(); __syncwarp(); };
         Step sx;
         for (int it = 0; it < n_it; ++it, sx.next(n_head)) {
           const int s = it % C::NS;
@@ -469,19 +481,23 @@ __global__ void __launch_bounds__(384, 1)
           float* dst = args.dq_acc + ((size_t)(bh * args.G + sx.g) * args.N_q + q_tile * 128) * D;
           // queries 0..63 (warpgroup 0), staged over the Q half; then 64..127 over the dO half
           if (!mbar_wait(bar_staged, it & 1, abort_flag, kSiteBwdDrain)) break;
-          bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows0 * D * 4));
-          bulk_commit();
-          bulk_wait_read0();
-          mbar_arrive(bar_q_empty(s));  // the producer may load the next Q here
-          if (!mbar_wait(bar_staged1, it & 1, abort_flag, kSiteBwdDrain)) break;
-          if (rows1 > 0) {
-            bulk_reduce_add_f32(dst + 64 * D, sDO(s), (uint32_t)(rows1 * D * 4));
+          one([&] {
+            bulk_reduce_add_f32(dst, sQ(s), (uint32_t)(rows0 * D * 4));
             bulk_commit();
             bulk_wait_read0();
-          }
-          mbar_arrive(bar_qb_empty(s));  // ... and the next dO here
+            mbar_arrive(bar_q_empty(s));  // the producer may load the next Q here
+          });
+          if (!mbar_wait(bar_staged1, it & 1, abort_flag, kSiteBwdDrain)) break;
+          one([&] {
+            if (rows1 > 0) {
+              bulk_reduce_add_f32(dst + 64 * D, sDO(s), (uint32_t)(rows1 * D * 4));
+              bulk_commit();
+              bulk_wait_read0();
+            }
+            mbar_arrive(bar_qb_empty(s));  // ... and the next dO here
+          });
         }
-        bulk_wait0();  // the last reduce has landed in global memory
+        one([&] { bulk_wait0(); });  // the last reduce has landed in global memory
       }
       __syncwarp();
     }

@@ -150,26 +150,33 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(bar_q_full, C::TILE);
+    // The whole warp runs the loop and its waits; lane 0 alone issues the copies
+    // and the barrier transactions (one()).
+    {
+      auto one = [&](auto f) { if (lane == 0) f(); __syncwarp(); };
+      one([&] {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        mbar_arrive_expect_tx(bar_q_full, C::TILE);
 #pragma unroll
-      for (int kb = 0; kb < C::L::NB; ++kb)
-        tma_load_3d(sQ + kb * C::L::BLKB, &tm_q, bar_q_full, kb * C::L::CW, rt * 128, hb);
+        for (int kb = 0; kb < C::L::NB; ++kb)
+          tma_load_3d(sQ + kb * C::L::BLKB, &tm_q, bar_q_full, kb * C::L::CW, rt * 128, hb);
+      });
       int it = 0;  // K_j at 2j, V_j at 2j + 1 (j counted from the split's first tile)
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
         for (int t = 0; t < 2 && ok; ++t, ++it) {
           const int s = it % C::NSLOT;
           if (!(ok = mbar_wait(bar_slot_empty(s), ((it / C::NSLOT) & 1) ^ 1, abort_flag, kSiteDecProducer))) break;
-          mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
-          const CUtensorMap* map = t == 0 ? &tm_k : &tm_v;
+          one([&] {
+            mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
+            const CUtensorMap* map = t == 0 ? &tm_k : &tm_v;
 #pragma unroll
-          for (int kb = 0; kb < C::L::NB; ++kb)
-            tma_load_3d(sSlot0 + s * C::TILE + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW,
-                        (j0 + j) * 128, hb);
+            for (int kb = 0; kb < C::L::NB; ++kb)
+              tma_load_3d(sSlot0 + s * C::TILE + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW,
+                          (j0 + j) * 128, hb);
+          });
         }
       }
       if (!ok) {  // aborted: let the copies already issued land before the CTA exits

@@ -168,17 +168,22 @@ __global__ void __launch_bounds__(384, 1)
     regs_decrease<56>();
     if (warp == 8) {
       // ---------------------------------------------------------- producer
-      if (lane == 0) {
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_do);
-        mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE);
+      // The whole warp runs the loop and its waits; lane 0 alone issues the copies
+      // and the barrier transactions (one()).
+      {
+        auto one = [&](auto f) { if (lane == 0) f(); __syncwarp(); };
+        one([&] {
+          prefetch_tensormap(&tm_q);
+          prefetch_tensormap(&tm_k);
+          prefetch_tensormap(&tm_v);
+          prefetch_tensormap(&tm_do);
+          mbar_arrive_expect_tx(bar_q_full, 2 * C::TILE);
 #pragma unroll
-        for (int kb = 0; kb < C::L::NB; ++kb) {
-          tma_load_3d(sQ + kb * C::L::BLKB, &tm_q, bar_q_full, kb * C::L::CW, q_tile * 128, bh);
-          tma_load_3d(sDO + kb * C::L::BLKB, &tm_do, bar_q_full, kb * C::L::CW, q_tile * 128, bh);
-        }
+          for (int kb = 0; kb < C::L::NB; ++kb) {
+            tma_load_3d(sQ + kb * C::L::BLKB, &tm_q, bar_q_full, kb * C::L::CW, q_tile * 128, bh);
+            tma_load_3d(sDO + kb * C::L::BLKB, &tm_do, bar_q_full, kb * C::L::CW, q_tile * 128, bh);
+          }
+        });
         int it = 0;  // tiles loaded: K_j at 2j, V_j at 2j + 1
         bool ok = true;
         for (int j = 0; j < n_kv && ok; ++j) {
@@ -186,12 +191,14 @@ __global__ void __launch_bounds__(384, 1)
             const int s = it % C::NSLOT;
             if (!(ok = mbar_wait(bar_slot_empty(s), ((it / C::NSLOT) & 1) ^ 1, abort_flag, kSiteDqProducer)))
               break;
-            mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
-            const CUtensorMap* map = t == 0 ? &tm_k : &tm_v;
+            one([&] {
+              mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
+              const CUtensorMap* map = t == 0 ? &tm_k : &tm_v;
 #pragma unroll
-            for (int kb = 0; kb < C::L::NB; ++kb)
-              tma_load_3d(sSlot0 + s * C::TILE + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW, j * 128,
-                          kv_bh);
+              for (int kb = 0; kb < C::L::NB; ++kb)
+                tma_load_3d(sSlot0 + s * C::TILE + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW, j * 128,
+                            kv_bh);
+            });
           }
         }
         if (!ok) {  // aborted: let the copies already issued land before the CTA exits

@@ -233,10 +233,16 @@ __global__ void __launch_bounds__(384, 1)
     regs_decrease<88>();
     if (warp == 8) {
       // ------------------------------------------------------------ producer
-      if (lane == 0) {
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
+      // The whole warp runs the loop and its waits; lane 0 alone issues the copies,
+      // the barrier transactions and the unit claims (one()).  A lone lane running
+      // the loop competes for issue slots with the softmax warps beside it.
+      {
+        auto one = [&](auto f) { if (lane == 0) f(); __syncwarp(); };
+        one([&] {
+          prefetch_tensormap(&tm_q);
+          prefetch_tensormap(&tm_k);
+          prefetch_tensormap(&tm_v);
+        });
         int it = 0;  // K/V tiles loaded (ring position), continuous across units
         int qs = 0;  // Q tiles loaded (Q ring position)
         bool ok = true;
@@ -244,8 +250,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int nu = 0; ok; ++nu) {
           const int e = nu % C::NUNIT;
           if (!(ok = mbar_wait(bar_unit_empty(e), ((nu / C::NUNIT) & 1) ^ 1, abort_flag, kSiteFwdUnit))) break;
-          unit_ring[e] = u < args.num_units ? u : -1;
-          mbar_arrive(bar_unit_full(e));
+          one([&] {
+            unit_ring[e] = u < args.num_units ? u : -1;
+            mbar_arrive(bar_unit_full(e));
+          });
           if (u >= args.num_units) break;
           const Unit w = unit_of(u);
           const int nq = w.n_kv1 > 0 ? 2 : 1;
@@ -254,28 +262,36 @@ __global__ void __launch_bounds__(384, 1)
             // A dynamic CTA claims its next unit as the loads of this unit's last
             // key/value tile go out: late enough that no CTA sits on a unit while
             // another has run out of work, early enough to hide the atomic.
-            if (dyn && j == w.n_kv - 1) ticket = atomicAdd(args.sched, 1u);
+            if (dyn && j == w.n_kv - 1) {
+              unsigned int t = 0;
+              if (lane == 0) t = atomicAdd(args.sched, 1u);
+              ticket = __shfl_sync(0xffffffffu, t, 0);
+            }
             for (int t = 0; t < 2 && ok; ++t) {
               const int s = it % C::NSLOT;
               if (!(ok = mbar_wait(bar_slot_empty(s), ((it / C::NSLOT) & 1) ^ 1, abort_flag, kSiteFwdProducer)))
                 break;
-              mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
-              const CUtensorMap* map = (t == 0) ? &tm_k : &tm_v;
-              const uint32_t dst = sSlot0 + s * C::TILE;
+              one([&] {
+                mbar_arrive_expect_tx(bar_slot_full(s), C::TILE);
+                const CUtensorMap* map = (t == 0) ? &tm_k : &tm_v;
+                const uint32_t dst = sSlot0 + s * C::TILE;
 #pragma unroll
-              for (int kb = 0; kb < C::L::NB; ++kb)
-                tma_load_3d(dst + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW, j * 128, w.kv_bh);
+                for (int kb = 0; kb < C::L::NB; ++kb)
+                  tma_load_3d(dst + kb * C::L::BLKB, map, bar_slot_full(s), kb * C::L::CW, j * 128, w.kv_bh);
+              });
               ++it;
               // Q0 after K_0, Q1 after V_0: each into the Q buffer freed longest ago
               if (j == 0 && t < nq) {
                 const int b = qs % C::QBUF;
                 if (!(ok = mbar_wait(bar_q_empty(b), ((qs / C::QBUF) & 1) ^ 1, abort_flag, kSiteFwdProducer)))
                   break;
-                mbar_arrive_expect_tx(bar_q_full(b), C::TILE);
+                one([&] {
+                  mbar_arrive_expect_tx(bar_q_full(b), C::TILE);
 #pragma unroll
-                for (int kb = 0; kb < C::L::NB; ++kb)
-                  tma_load_3d(sQ(b) + kb * C::L::BLKB, &tm_q, bar_q_full(b), kb * C::L::CW, (w.tile0 + t) * 128,
-                              w.bh);
+                  for (int kb = 0; kb < C::L::NB; ++kb)
+                    tma_load_3d(sQ(b) + kb * C::L::BLKB, &tm_q, bar_q_full(b), kb * C::L::CW, (w.tile0 + t) * 128,
+                                w.bh);
+                });
                 ++qs;
               }
             }
