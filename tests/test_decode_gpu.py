@@ -43,6 +43,9 @@ CASES = [
     (1, 4, 4, 5, 1000, 1024, 64, 3),       # ragged cache, five new rows
     (1, 32, 1, 8, 2048, 2048, 128, 0),     # 256 packed rows: two row tiles
     (3, 6, 3, 16, 777, 800, 64, 0),        # sixteen new rows, ragged
+    (1, 8, 2, 1, 3000, 3072, 256, 0),      # d = 256, library-chosen splits, ragged cache
+    (2, 4, 1, 3, 1500, 1600, 96, 0),       # d = 96, one key/value head, three new rows
+    (1, 6, 3, 2, 2500, 2500, 32, 4),       # d = 32, four splits
 ]
 
 
