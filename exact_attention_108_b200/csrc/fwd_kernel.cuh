@@ -102,7 +102,19 @@ struct FwdCfg {
   static constexpr int TM_O = 256;                     // O_k at 256 + k * D
 };
 
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: weights stay below 256
+constexpr float kRescaleThreshold = 8.0f;
+// A quarter of the unmasked tiles' exponentials (2 of every 8 pairs) run on the
+// FMA pipe instead of MUFU, which the softmax's exponentials otherwise keep busy
+// about as long as the tensor cores run a tile's products.  2^x = 2^n 2^f with
+// n = round(x), f = x - n in [-1/2, 1/2] (Cody-Waite reduction), 2^f by a cubic
+// whose coefficients minimise the relative error on [-1/2, 1/2] with p(0) = 1
+// (fit_exp2_poly.py, a linear programme; largest relative error 1.013e-4, far
+// below the bf16 rounding of P).  x is first clamped to [-124, 132] through a
+// saturated y = (x + 124) / 256, so that adding n to the exponent field of 2^f
+// never leaves the normal range; clamping at -124 turns weights below 2^-124
+// (invisible next to a row's largest, which is at least 2^-8) into 2^-124.
+constexpr int kFmaPairsPer8 = 2;
+constexpr float kExpC1 = 0.6932829022407532f, kExpC2 = 0.2422109693288803f, kExpC3 = 0.055009059607982635f;  // log2 units: weights stay below 256
 
 enum : int {  // wait sites recorded in the device status word on a timeout
   kSiteFwdProducer = 0x101,
@@ -532,6 +544,7 @@ __global__ void __launch_bounds__(384, 1)
         // copy tests the mask per element (a second copy would spill).
         const uint32_t q_row = (uint32_t)(q_tile * 128 + r);
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
+        const float pa = sl2 * (1.f / 256.f), pb = (124.f - m_ref) * (1.f / 256.f);  // y = s pa + pb
         uint32_t pk[2][32];  // P row as packed bf16 pairs
         auto exps = [&](auto mode_c) {
           constexpr int MODE = decltype(mode_c)::value;  // 0: no mask, 1: mask, 2: mask if clip
@@ -542,9 +555,29 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(v[c >> 5][c & 31]),
                                                __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31])),
                                        sl2x2, negm2);
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            float p0 = ex2(x0), p1 = ex2(x1);
+            float p0, p1;
+            if (MODE == 0 && ((c >> 1) & 7) < kFmaPairsPer8) {
+              // y = sat((x + 124) / 256) stands for x; t = 1.5 * 2^23 + round(x) carries n
+              // in its low bits; f = x - n; 2^f by the cubic; n added to the exponent
+              const uint64_t y = f2_pack(fma_sat(__uint_as_float(v[c >> 5][c & 31]), pa, pb),
+                                         fma_sat(__uint_as_float(v[(c + 1) >> 5][(c + 1) & 31]), pa, pb));
+              const uint64_t t = f2_fma(y, f2_pack(256.f, 256.f), f2_pack(12582912.f - 124.f, 12582912.f - 124.f));
+              const uint64_t w2 = f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(12582912.f - 124.f, 12582912.f - 124.f));
+              const uint64_t f = f2_fma(y, f2_pack(256.f, 256.f), w2);
+              uint64_t q = f2_fma(f, f2_pack(kExpC3, kExpC3), f2_pack(kExpC2, kExpC2));
+              q = f2_fma(q, f, f2_pack(kExpC1, kExpC1));
+              q = f2_fma(q, f, f2_pack(1.f, 1.f));
+              float q0, q1, t0, t1;
+              f2_unpack(q, q0, q1);
+              f2_unpack(t, t0, t1);
+              p0 = __uint_as_float(imad_u32(__float_as_uint(t0), 1u << 23, __float_as_uint(q0)));
+              p1 = __uint_as_float(imad_u32(__float_as_uint(t1), 1u << 23, __float_as_uint(q1)));
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
             if (MODE == 1 || (MODE == 2 && clip)) {
               p0 = (c < lim) ? p0 : 0.f;
               p1 = (c + 1 < lim) ? p1 : 0.f;
